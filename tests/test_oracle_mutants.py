@@ -1,0 +1,44 @@
+"""Plant plausible mistakes in a copy of the oracle (on the CPU) and check
+that the pins catch every one of them."""
+
+import os
+import shutil
+
+import pytest
+
+import oracle
+import _oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+# (name, exact text in oracle.c, replacement)
+MUTANTS = [
+    ("drop_scale", "s[j] = J->scale * dot;", "s[j] = dot;"),
+    ("causal_off_by_one", "if (J->causal && (long)j > (long)i", "if (J->causal && (long)j >= (long)i"),
+    ("causal_top_left", "(long)i + (long)J->Nk - (long)J->Nq", "(long)i"),
+    ("gqa_modulo", "const int hk = hq / group;", "const int hk = hq % J->Hkv;"),
+    ("no_max_in_lse", "*lse_out = m + log(l);", "*lse_out = log(l);"),
+    ("no_division", "orow[c] /= l;", "orow[c] /= 1.0;"),
+    ("v_from_k", "const uint16_t *vrow = J->v +", "const uint16_t *vrow = J->k +"),
+    ("max_not_subtracted_in_weights", "s[j] = exp(s[j] - m);", "s[j] = exp(s[j] - m * 0.5);"),
+    ("ignore_key_range", "if (j < J->k_begin || j >= J->k_end)", "if (0)"),
+    ("q_row_index", "(((size_t)b * J->Nq + i) * J->Hq + hq) * d;", "(((size_t)b * J->Nq + ri) * J->Hq + hq) * d;"),
+    ("drop_one_key_term", "for (int c = 0; c < d; ++c)\n            dot += qd[c]", "for (int c = 1; c < d; ++c)\n            dot += qd[c]"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, name, old, new):
+    text = open(SRC).read()
+    assert text.count(old) == 1, f"mutation site for {name} not found exactly once"
+    src = tmp_path / "oracle_mut.c"
+    src.write_text(text.replace(old, new))
+    so = oracle.build(force=True, src=str(src), out=str(tmp_path / "liboracle_mut.so"))
+    orc = oracle.Oracle(so)
+    failed = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(orc)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, f"mutant {name} passed every pin"

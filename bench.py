@@ -1,0 +1,396 @@
+#!/usr/bin/env python3
+"""Benchmark of the B200 attention forward pass; prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload causal_8k] [--impl fa2|reference]
+
+A step is one forward pass (one launch of the CUDA kernel) over the workload's
+synthetic inputs, already resident in HBM.  L2 is flushed (a 256 MiB write)
+before every step, outside the per-step CUDA events that time the launch on
+its own stream.  ``value`` = algorithmic TFLOP/s of all ranks (4*B*Hq*Nq*Nk*d,
+halved when causal) / max-over-ranks mean step time.  With N > 1 (torchrun),
+each rank runs its own independently seeded batch of the same workload (weak
+scaling; the ranks exchange nothing but the timing reduction).
+
+``e2e`` measures the same metric through the public API with host buffers:
+pinned-host Q/K/V -> device, the C-ABI call, O and LSE -> pinned host.
+``--impl reference`` times the CPU fp64 oracle on a bounded sample instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_tiled_attention_29_b200.inputs import WORKLOADS, bf16_bits, make_qkv  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s (bf16, 1 B200) and % of dense BF16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SRC = os.path.join(ROOT, "exact_tiled_attention_29_b200", "csrc", "fa2_forward.cu")
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="causal_8k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="fa2", choices=["fa2", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in (KERNEL_SRC, os.path.join(ROOT, "exact_tiled_attention_29_b200", "csrc", "sm100_ptx.cuh")):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"fa2_fwd_kernel_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_h = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m_b or not m_h or m_h.group(1) != kernel_source_hash():
+        return None
+    return float(m_b.group(1))
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    """Samples nvidia-smi clocks/throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self._thr = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self._thr = threading.Thread(target=self._read, daemon=True)
+        self._thr.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self._thr:
+            self._thr.join(timeout=2)
+        return self.summary()
+
+    def summary(self):
+        mhz, maxmhz, power, reasons = [], None, [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for _, line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                maxmhz = float(parts[2])
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() in ("active", "1", "yes"):
+                    reasons.add(n)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": maxmhz, "reasons": sorted(reasons),
+                "samples": len(mhz), "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------- CPU arm --
+
+def oracle_sample_rows(w, seconds: float, orc, q, k, v):
+    """Pick evenly spaced rows of head (b=0, all heads) so the oracle runs for ~`seconds`."""
+    import numpy as np
+    # calibrate on a handful of rows spread over the sequence
+    cal = np.linspace(0, w.Nq - 1, 16).astype(np.int32)
+    t0 = time.perf_counter()
+    orc.attention(q, k, v, w.causal, w.softmax_scale, rows=cal)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    per_row = dt / (len(cal) * w.B * w.Hq)
+    n = int(max(8, min(w.Nq, seconds / per_row / (w.B * w.Hq))))
+    return np.unique(np.linspace(0, w.Nq - 1, n).astype(np.int32))
+
+
+def sample_flops(w, rows) -> float:
+    vis = [(min(int(r) + w.Nk - w.Nq, w.Nk - 1) + 1) if w.causal else w.Nk for r in rows]
+    vis = [max(0, x) for x in vis]
+    return 4.0 * w.d * w.B * w.Hq * float(sum(vis))
+
+
+def cpu_oracle_baseline(w, seconds: float):
+    import oracle
+    orc = oracle._get()
+    q, k, v = (bf16_bits(t) for t in make_qkv(w))
+    rows = oracle_sample_rows(w, seconds, orc, q, k, v)
+    t0 = time.perf_counter()
+    orc.attention(q, k, v, w.causal, w.softmax_scale, rows=rows)
+    dt = time.perf_counter() - t0
+    fl = sample_flops(w, rows)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": orc.default_threads(),
+            "kind": "oracle",
+            "sample": f"{len(rows)} evenly spaced query rows x all {w.B * w.Hq} (batch, head) pairs "
+                      f"of {w.name}, every visible key, fp64 C oracle; {fl:.3g} algorithmic FLOP in "
+                      f"{dt:.2f} s"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    orc = oracle._get()
+    q, k, v = (bf16_bits(t) for t in make_qkv(w))
+    per_step = max(0.02, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    rows = oracle_sample_rows(w, per_step, orc, q, k, v)
+    fl = sample_flops(w, rows)
+    for _ in range(args.warmup):
+        orc.attention(q, k, v, w.causal, w.softmax_scale, rows=rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.attention(q, k, v, w.causal, w.softmax_scale, rows=rows)
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
+    val = fl / dt / 1e12
+    sample = (f"{len(rows)} evenly spaced query rows x all {w.B * w.Hq} (batch, head) pairs of "
+              f"{w.name} per step, every visible key, fp64 C oracle")
+    line = {"metric": METRIC, "value": val, "unit": "TFLOP/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, args.gpus),
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": orc.default_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, n_gpus):
+    return {"workload": w.name, "description": w.description, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+            "Nq": w.Nq, "Nk": w.Nk, "d": w.d, "causal": w.causal,
+            "softmax_scale": w.softmax_scale, "seed": w.seed,
+            "flops_per_step_per_rank": w.flops(),
+            "parallelism": f"independent batches per rank x{n_gpus}" if n_gpus > 1 else "single GPU",
+            "l2": "flushed before every step (256 MiB write), outside the per-step events"}
+
+
+# ---------------------------------------------------------------- GPU arm --
+
+def run_fa2(args, w):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    import exact_tiled_attention_29_b200 as fa2
+
+    q_h, k_h, v_h = make_qkv(w, seed=w.seed + rank)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def forward():
+        st = fa2.fa2_forward(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
+                             w.softmax_scale, stream)
+        if st != 0:
+            raise fa2.FA2Error(st)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        forward()
+    torch.cuda.synchronize()
+    dstat = fa2.fa2_debug_status(stream)
+    if dstat != 0:
+        raise RuntimeError(f"device status {dstat:#x} after warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_all0 = torch.cuda.Event(enable_timing=True)
+    t_all1 = torch.cuda.Event(enable_timing=True)
+    t_all0.record(stream)
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        forward()
+        ends[i].record(stream)
+    t_all1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    mean_ms = sum(step_ms) / len(step_ms)
+    bracket_ms = t_all0.elapsed_time(t_all1)
+    dstat = fa2.fa2_debug_status(stream)
+    if dstat != 0:
+        raise RuntimeError(f"device status {dstat:#x} after the timed region")
+
+    if world > 1:
+        t = torch.tensor([mean_ms, bracket_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        mean_ms, bracket_ms = float(t[0]), float(t[1])
+
+    # ---- end-to-end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        qp, kp, vp = (t.pin_memory() for t in (q_h, k_h, v_h))
+        op = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        lp = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        od, ld = torch.empty_like(o), torch.empty_like(lse)
+        n_e2e = max(3, min(args.steps, 50))
+
+        def e2e_step():
+            qd.copy_(qp, non_blocking=True)
+            kd.copy_(kp, non_blocking=True)
+            vd.copy_(vp, non_blocking=True)
+            st = fa2.fa2_forward(qd, kd, vd, od, ld, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
+                                 w.softmax_scale, stream)
+            if st != 0:
+                raise fa2.FA2Error(st)
+            op.copy_(od, non_blocking=True)
+            lp.copy_(ld, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / n_e2e
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t[0])
+        if not torch.isfinite(lp).any():
+            raise RuntimeError("e2e produced no finite LSE")
+        h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
+        d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+        e2e = {"value": world * w.flops() / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": n_e2e}
+
+    value = world * w.flops() / (mean_ms * 1e-3) / 1e12
+    line = None
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        peak = float(peaks["bf16_tflops"])
+        achieved = w.flops() / (mean_ms * 1e-3) / 1e12
+        traffic = profiled_traffic(w.name)
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_oracle_baseline(w, args.cpu_seconds)
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(w, world),
+            "pct_of_peak": 100.0 * achieved / peak,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"bf16_tflops (burst, kernel timed alone), {peak_src}",
+                         "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"]),
+                         "kernel": "fa2_fwd_kernel<128>" if w.d == 128 else "fa2_fwd_kernel<64>"},
+            "hbm_gbs_compulsory": w.compulsory_bytes() / (mean_ms * 1e-3) / 1e9,
+            "bracket_ms_per_step_incl_flush": bracket_ms / args.steps,
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "kernel_source_sha256_16": kernel_source_hash(),
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_fa2(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

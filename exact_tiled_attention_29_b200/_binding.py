@@ -1,0 +1,140 @@
+"""ctypes binding of ``libfa2.so`` (the C ABI declared in ``include/fa2.h``).
+
+Argument marshalling only: every step of the attention forward pass runs in
+the CUDA library.  Importing this module loads the in-tree library and raises
+``ImportError`` if it is missing -- there is no fallback implementation.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa2.so")
+
+FA2_OK = 0
+STATUS_NAMES = {
+    0: "FA2_OK", 1: "FA2_ERR_NULL_POINTER", 2: "FA2_ERR_BAD_SHAPE", 3: "FA2_ERR_HEAD_DIM",
+    4: "FA2_ERR_ALIGNMENT", 5: "FA2_ERR_SCALE", 6: "FA2_ERR_DEVICE", 7: "FA2_ERR_LAUNCH",
+    8: "FA2_ERR_SIZE", 9: "FA2_ERR_BUILD",
+}
+SITE_NAMES = {
+    1: "Q_LOADED", 2: "KV_LOADED", 3: "KV_FREE", 4: "S_READY", 5: "P_READY", 6: "STATS_READY",
+    7: "O_RESCALED", 8: "O_FINAL", 9: "FINAL_STATS", 10: "MMA_DRAIN", 11: "LOAD_DRAIN",
+    15: "SELFTEST",
+}
+FA2_SITE_SELFTEST = 15
+
+
+class FA2Error(RuntimeError):
+    def __init__(self, status: int, where: str = "fa2_forward"):
+        self.status = status
+        super().__init__(f"{where} failed with status {status} ({fa2_status_string(status)})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m exact_tiled_attention_29_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, ci, cf, cll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
+    lib.fa2_forward.argtypes = [vp, vp, vp, vp, vp] + [ci] * 7 + [cf, vp]
+    lib.fa2_forward.restype = ci
+    lib.fa2_status_string.argtypes = [ci]
+    lib.fa2_status_string.restype = ctypes.c_char_p
+    lib.fa2_debug_status.argtypes = [vp]
+    lib.fa2_debug_status.restype = ci
+    lib.fa2_selftest_timeout.argtypes = [vp, cll]
+    lib.fa2_selftest_timeout.restype = ci
+    lib.fa2_num_blocks.argtypes = [ci, ci, ci, ci]
+    lib.fa2_num_blocks.restype = cll
+    ip = ctypes.POINTER(ci)
+    lib.fa2_launch_plan.argtypes = [ci] * 6 + [ip] * 4
+    lib.fa2_launch_plan.restype = ci
+    return lib
+
+
+_lib = _load()
+
+
+def _ptr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return int(x.data_ptr())
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return int(s.cuda_stream)
+
+
+# ---- the C ABI, one function per entry point, same names ----
+
+def fa2_forward(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, stream) -> int:
+    """Enqueue the forward pass; pointers may be ints or tensors.  Returns the status code."""
+    return int(_lib.fa2_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(Hq),
+                                int(Hkv), int(Nq), int(Nk), int(d), int(bool(causal)),
+                                float(softmax_scale), _stream(stream)))
+
+
+def fa2_status_string(status: int) -> str:
+    return _lib.fa2_status_string(int(status)).decode()
+
+
+def fa2_debug_status(stream=None) -> int:
+    return int(_lib.fa2_debug_status(_stream(stream)))
+
+
+def fa2_selftest_timeout(stream, limit_ns: int) -> int:
+    return int(_lib.fa2_selftest_timeout(_stream(stream), int(limit_ns)))
+
+
+def fa2_num_blocks(B: int, H: int, N: int, rows_per_block: int) -> int:
+    return int(_lib.fa2_num_blocks(int(B), int(H), int(N), int(rows_per_block)))
+
+
+def fa2_launch_plan(B, Hq, Hkv, Nq, Nk, d):
+    """(status, grid_blocks, threads_per_block, smem_bytes, rows_per_block)."""
+    out = [ctypes.c_int(0) for _ in range(4)]
+    st = _lib.fa2_launch_plan(int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
+                              *[ctypes.byref(x) for x in out])
+    return (int(st), *[x.value for x in out])
+
+
+# ---- torch convenience: allocate outputs with torch, then call the C ABI ----
+
+def attention(q, k, v, causal: bool = False, softmax_scale: float | None = None, out=None,
+              lse=None, stream=None):
+    """O, LSE for bf16 CUDA tensors q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d] (contiguous).
+
+    Outputs are allocated with torch unless given; the work is one call to
+    ``fa2_forward`` on ``stream`` (default: torch's current stream).
+    """
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D bf16 CUDA tensor")
+    B, Nq, Hq, d = q.shape
+    Bk, Nk, Hkv, dk = k.shape
+    if v.shape != k.shape or Bk != B or dk != d:
+        raise ValueError("k and v must be [B, Nk, Hkv, d] with q's B and d")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    st = fa2_forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, stream)
+    if st != FA2_OK:
+        raise FA2Error(st)
+    return out, lse

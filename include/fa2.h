@@ -1,0 +1,132 @@
+/*
+ * fa2.h -- C ABI of the B200 (sm_100a) exact attention forward pass.
+ *
+ * The library computes, for every batch b, query head hq and query row i,
+ *
+ *     O[b,i,hq,:] = softmax_j( softmax_scale * q[b,i,hq,:] . k[b,j,hk,:] ) v[b,j,hk,:]
+ *     LSE[b,hq,i] = ln sum_j exp( softmax_scale * q[b,i,hq,:] . k[b,j,hk,:] )
+ *
+ * over the keys j visible to row i, exactly (up to floating-point rounding):
+ * the result of standard attention, computed tile by tile with a running row
+ * maximum and denominator so the Nq x Nk score matrix never exists in memory.
+ * Sources: "FlashAttention 2: Three Places the Chip Was Still Waiting",
+ * section 1 ("New here?": tiling and online softmax, the answer is exact) and
+ * section 2.2 (the accumulator stays unnormalised and is divided once per
+ * query block); "FlashAttention-2 and -3: From Algebra to GPU Scheduling",
+ * "Keep the unchanged mathematical target in view".
+ *
+ * Conventions the pages leave open, fixed here:
+ *   - causal: key j is visible to query row i iff j <= i + (Nk - Nq)
+ *     (bottom-right alignment; the usual j <= i when Nq == Nk);
+ *   - GQA ("GQA-aware" variants, "FlashAttention-2" explainer, "The
+ *     Downstream Story"): query head hq reads KV head hq / (Hq / Hkv), i.e.
+ *     consecutive groups of Hq/Hkv query heads share one KV head;
+ *   - a row with no visible key gets O = 0 and LSE = -inf;
+ *   - LSE is the natural log and includes softmax_scale.
+ *
+ * All entry points are thread-safe and allocate no device memory.
+ */
+#ifndef FA2_H
+#define FA2_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by the host entry points. */
+enum fa2_status_code {
+  FA2_OK = 0,
+  FA2_ERR_NULL_POINTER = 1,   /* a required pointer is NULL                          */
+  FA2_ERR_BAD_SHAPE = 2,      /* B, Hq, Hkv, Nq or Nk <= 0, or Hq % Hkv != 0         */
+  FA2_ERR_HEAD_DIM = 3,       /* d is not 64 or 128                                  */
+  FA2_ERR_ALIGNMENT = 4,      /* q, k, v, o not 16-byte aligned, or lse not 4-byte   */
+  FA2_ERR_SCALE = 5,          /* softmax_scale is NaN or infinite                    */
+  FA2_ERR_DEVICE = 6,         /* current device is not compute capability 10.0      */
+  FA2_ERR_LAUNCH = 7,         /* a CUDA runtime/driver call or the launch failed    */
+  FA2_ERR_SIZE = 8,           /* a tensor or the grid exceeds the supported extent   */
+  FA2_ERR_BUILD = 9           /* the kernel image does not match its register plan  */
+};
+
+/*
+ * fa2_forward -- enqueue one attention forward pass on `stream`.
+ *
+ *   q    device pointer, bf16 [B, Nq, Hq,  d], contiguous (d fastest); read only
+ *   k    device pointer, bf16 [B, Nk, Hkv, d], contiguous; read only
+ *   v    device pointer, bf16 [B, Nk, Hkv, d], contiguous; read only
+ *   o    device pointer, bf16 [B, Nq, Hq,  d], contiguous; written (every element)
+ *   lse  device pointer, fp32 [B, Hq, Nq],     contiguous; written (every element)
+ *   B, Hq, Hkv, Nq, Nk   sizes, all > 0, Hq a multiple of Hkv
+ *   d               head dimension, 64 or 128
+ *   causal          0 = every key visible, nonzero = causal (see above)
+ *   softmax_scale   any finite value (1/sqrt(d) is the usual choice)
+ *   stream          cudaStream_t to launch on; NULL = the legacy default stream
+ *
+ * Ownership: the caller owns every buffer; the library keeps no reference after
+ * the call returns.  o and lse must not overlap q, k or v (undefined otherwise).
+ * The call is asynchronous: it validates the arguments (before any CUDA call,
+ * so validation works without a GPU), builds the TMA descriptors, launches one
+ * kernel and returns.  Errors are returned as fa2_status_code values; nothing
+ * is thrown across the ABI.  A kernel that gave up on a wait (a bounded wait
+ * that ran out; never expected in normal operation) leaves a nonzero code that
+ * fa2_debug_status reports.
+ */
+int fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                int Hkv, int Nq, int Nk, int d, int causal, float softmax_scale, void* stream);
+
+/* Human-readable text for a status code (static storage, never NULL). */
+const char* fa2_status_string(int status);
+
+/*
+ * fa2_debug_status -- synchronise `stream`, return the device status word of
+ * the current device and reset it to 0.  0 means no kernel gave up on a wait;
+ * otherwise the value is (site << 16) | (iteration & 0xffff), where site
+ * names the wait (FA2_SITE_* below).  Returns -1 if a CUDA call failed.
+ */
+int fa2_debug_status(void* stream);
+
+/* Wait sites reported by fa2_debug_status. */
+enum fa2_wait_site {
+  FA2_SITE_Q_LOADED = 1,
+  FA2_SITE_KV_LOADED = 2,
+  FA2_SITE_KV_FREE = 3,
+  FA2_SITE_S_READY = 4,
+  FA2_SITE_P_READY = 5,
+  FA2_SITE_STATS_READY = 6,
+  FA2_SITE_O_RESCALED = 7,
+  FA2_SITE_O_FINAL = 8,
+  FA2_SITE_FINAL_STATS = 9,
+  FA2_SITE_MMA_DRAIN = 10,
+  FA2_SITE_LOAD_DRAIN = 11,
+  FA2_SITE_SELFTEST = 15
+};
+
+/*
+ * fa2_selftest_timeout -- launch a one-warp kernel that waits on an mbarrier
+ * nothing ever arrives on, with the given limit in nanoseconds (1 ms .. 10 s),
+ * through the same bounded-wait routine the attention kernel uses.  The wait
+ * runs out, the kernel records FA2_SITE_SELFTEST and returns; read it with
+ * fa2_debug_status.  Exercises the failure path without faulting the GPU.
+ */
+int fa2_selftest_timeout(void* stream, long long limit_ns);
+
+/*
+ * Host-only planning helpers (no CUDA calls).
+ *
+ * fa2_num_blocks: thread blocks of a grid that runs over (query tile, head,
+ * batch), ceil(N / rows_per_block) * H * B -- the sequence-parallel grid of
+ * "FlashAttention 2: Three Places the Chip Was Still Waiting", section 2.3.
+ * Returns -1 on non-positive arguments.
+ *
+ * fa2_launch_plan: the launch this library uses for a problem: grid size,
+ * threads per block, dynamic shared memory bytes and query rows per block.
+ * Returns an fa2_status_code (validation as in fa2_forward, minus pointers).
+ */
+long long fa2_num_blocks(int B, int H, int N, int rows_per_block);
+int fa2_launch_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int* grid_blocks,
+                    int* threads_per_block, int* smem_bytes, int* rows_per_block);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA2_H */

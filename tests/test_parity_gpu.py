@@ -1,0 +1,172 @@
+"""GPU forward pass vs the fp64 oracle, element by element, through the C ABI.
+
+Tolerances (on every compared row): O max-abs <= 2e-2 and mean-abs <= 2e-3,
+LSE max-abs <= 1e-3, no NaN/Inf where the oracle is finite.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_tiled_attention_29_b200.inputs import WORKLOADS, Workload, bf16_bits, make_qkv, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+O_MAX, O_MEAN, LSE_MAX = 2e-2, 2e-3, 1e-3
+
+
+@pytest.fixture(scope="module")
+def fa2():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import exact_tiled_attention_29_b200 as m
+    return m
+
+
+def run_gpu(fa2, q, k, v, causal, scale, guard=0):
+    """Run the C-ABI forward on copies of q, k, v; O and LSE are carved out of
+    NaN-filled buffers with `guard` poisoned elements on both sides."""
+    dev = torch.device("cuda")
+    qd, kd, vd = (t.to(dev).contiguous() for t in (q, k, v))
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    g_o = guard * d  # keep 16-byte alignment of the O view
+    o_buf = torch.full((B * Nq * Hq * d + 2 * g_o,), float("nan"), dtype=torch.bfloat16, device=dev)
+    l_buf = torch.full((B * Hq * Nq + 2 * max(guard, 4),), float("nan"), dtype=torch.float32, device=dev)
+    gl = max(guard, 4)
+    o = o_buf[g_o:g_o + B * Nq * Hq * d].view(B, Nq, Hq, d)
+    lse = l_buf[gl:gl + B * Hq * Nq].view(B, Hq, Nq)
+    st = fa2.fa2_forward(qd, kd, vd, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale,
+                         torch.cuda.current_stream())
+    assert st == 0, fa2.fa2_status_string(st)
+    torch.cuda.synchronize()
+    assert fa2.fa2_debug_status(None) == 0
+    if guard:
+        assert torch.isnan(o_buf[:g_o].float()).all() and torch.isnan(o_buf[-g_o:].float()).all(), \
+            "O guard band overwritten"
+    assert torch.isnan(l_buf[:gl]).all() and torch.isnan(l_buf[-gl:]).all(), "LSE guard band overwritten"
+    return o.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def compare(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
+    """o_* [B,R,Hq,d], lse_* [B,Hq,R] on the same rows."""
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isneginf(lse_gpu), np.isneginf(lse_ref)), f"{what}: -inf pattern of LSE"
+    assert np.isfinite(o_gpu).all(), f"{what}: non-finite O"
+    assert not np.isnan(lse_gpu).any(), f"{what}: NaN LSE"
+    err = np.abs(o_gpu - o_ref)
+    assert err.max() <= O_MAX, f"{what}: O max-abs {err.max():.3g}"
+    assert err.mean() <= O_MEAN, f"{what}: O mean-abs {err.mean():.3g}"
+    if fin.any():
+        lerr = np.abs(lse_gpu[fin] - lse_ref[fin]).max()
+        assert lerr <= LSE_MAX, f"{what}: LSE max-abs {lerr:.3g}"
+    return float(err.max()), float(err.mean())
+
+
+def check_case(fa2, w: Workload, rows=None, scale=None, guard=0):
+    q, k, v = make_qkv(w)
+    scale = w.softmax_scale if scale is None else scale
+    o_gpu, lse_gpu = run_gpu(fa2, q, k, v, w.causal, scale, guard=guard)
+    o_ref, lse_ref = oracle.attention(bf16_bits(q), bf16_bits(k), bf16_bits(v), w.causal, scale,
+                                      rows=rows)
+    if rows is not None:
+        o_gpu, lse_gpu = o_gpu[:, rows], lse_gpu[:, :, rows]
+    return compare(o_gpu, lse_gpu, o_ref, lse_ref, what=w.name)
+
+
+# ---- the five specified workloads, in the launch configuration the benchmark times ----
+
+def test_tiny_all_rows(fa2):
+    check_case(fa2, WORKLOADS["tiny"], guard=8)
+
+
+def test_noncausal_2k_all_rows(fa2):
+    check_case(fa2, WORKLOADS["noncausal_2k"])
+
+
+@pytest.mark.parametrize("name", ["causal_8k", "long_32k", "gqa_4k"])
+def test_full_size_sampled_rows(fa2, name):
+    w = WORKLOADS[name]
+    idx = list(WORKLOADS).index(name)
+    rows = sample_rows(w, 1024, seed=idx)
+    check_case(fa2, w, rows=rows)
+
+
+# ---- ragged and odd sizes, both head dims, Nq != Nk in both directions ----
+
+ODD = [1, 17, 127, 129, 1000]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("nq,nk", [(n, n) for n in ODD] + [(17, 1000), (1000, 17), (129, 127),
+                                                            (127, 129), (1, 1000), (300, 1)])
+def test_odd_sizes(fa2, d, causal, nq, nk):
+    w = Workload(f"odd{nq}x{nk}", 2, 4, 2, nq, nk, d, causal, seed=nq * 7 + nk)
+    check_case(fa2, w, guard=8)
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.0883883, 0.5])
+def test_scale_values(fa2, scale):
+    w = Workload("scale", 1, 2, 1, 300, 300, 128, True, seed=3)
+    check_case(fa2, w, scale=scale)
+
+
+def test_large_scores_outliers_d64(fa2):
+    w = Workload("outl64", 1, 2, 2, 2048, 2048, 64, True, seed=5, outlier_frac=0.01, outlier_scale=8.0)
+    check_case(fa2, w)
+
+
+# ---- closed forms on the GPU ----
+
+def test_causal_row0_is_v0_bitwise(fa2):
+    w = Workload("row0", 2, 4, 2, 384, 384, 128, True, seed=9)
+    q, k, v = make_qkv(w)
+    o, lse = run_gpu(fa2, q, k, v, True, w.softmax_scale)
+    vv = v.float().numpy()
+    for hq in range(4):
+        assert np.array_equal(o[:, 0, hq], vv[:, 0, hq // 2]), "row 0 must be exactly V[0]"
+    qk = np.einsum("bhc,bhc->bh", q.double().numpy()[:, 0], np.repeat(k.double().numpy()[:, 0], 2, axis=1))
+    assert np.abs(lse[:, :, 0] - w.softmax_scale * qk).max() < 1e-3
+
+
+def test_zero_query_gives_mean_of_visible_v(fa2):
+    w = Workload("q0", 1, 2, 2, 260, 260, 64, True, seed=10)
+    q, k, v = make_qkv(w)
+    q = torch.zeros_like(q)
+    o, lse = run_gpu(fa2, q, k, v, True, w.softmax_scale)
+    vv = v.double().numpy()
+    csum = np.cumsum(vv, axis=1) / np.arange(1, 261)[None, :, None, None]
+    assert np.abs(o - csum).max() < 2e-2
+    assert np.abs(lse - np.log(np.arange(1, 261))[None, None, :]).max() < 1e-3
+
+
+# ---- structural properties ----
+
+def test_gqa_equals_repeated_heads_bitwise(fa2):
+    w = Workload("gqa", 2, 8, 2, 700, 700, 128, True, seed=12)
+    q, k, v = make_qkv(w)
+    o1, l1 = run_gpu(fa2, q, k, v, True, w.softmax_scale)
+    o2, l2 = run_gpu(fa2, q, k.repeat_interleave(4, dim=2), v.repeat_interleave(4, dim=2), True,
+                     w.softmax_scale)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_deterministic_across_runs(fa2):
+    w = Workload("det", 2, 4, 4, 1500, 1500, 128, True, seed=13)
+    q, k, v = make_qkv(w)
+    outs = [run_gpu(fa2, q, k, v, True, w.softmax_scale) for _ in range(3)]
+    for o, l in outs[1:]:
+        assert np.array_equal(o, outs[0][0]) and np.array_equal(l, outs[0][1])
+
+
+def test_torch_convenience_wrapper(fa2):
+    w = Workload("wrap", 1, 4, 2, 333, 444, 64, False, seed=14)
+    q, k, v = make_qkv(w)
+    o, lse = fa2.attention(q.cuda(), k.cuda(), v.cuda(), causal=False)
+    torch.cuda.synchronize()
+    o_ref, l_ref = oracle.attention(bf16_bits(q), bf16_bits(k), bf16_bits(v), False, w.softmax_scale)
+    compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, what="wrapper")

@@ -222,15 +222,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kBlockN; ++i)
           if (i > lim) s[i] = -INFINITY;
       }
-      // row max as 8 independent chains (max is exact in any order)
+      // row max: 8 independent chains of 3-input max (max is exact in any order)
       float mp[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mp[i] = s[i];
+      for (int k = 0; k < 8; ++k) mp[k] = fmaxf(s[2 * k], s[2 * k + 1]);
 #pragma unroll
-      for (int i = 8; i < kBlockN; ++i) mp[i & 7] = fmaxf(mp[i & 7], s[i]);
-      float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                       fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      mx = fmaxf(mx, m_raw);
+      for (int i = 16; i < kBlockN; i += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mp[k] = fmax3(mp[k], s[i + 2 * k], s[i + 2 * k + 1]);
+      const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]),
+                             fmax3(mp[6], mp[7], m_raw));
       const float m_sc_new = (mx == -INFINITY) ? 0.f : mx * c;
       // rescale factor for what was accumulated so far: exactly 1 when the max
       // did not move (then O is left untouched), 0 when nothing was visible yet
@@ -242,8 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm_alpha[t * kBlockM + rt] = alpha;
         mbar_arrive(bar(BAR_STATS + t));
       }
-      const float neg = -m_sc_new;
-      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      // p = 2^(s*c - m*c): one packed FMA per pair of scores, then ex2
+      const uint64_t cc = f2_pack(c, c), nn = f2_pack(-m_sc_new, -m_sc_new);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // packed partial row sums (+0.0f pairs)
       const uint32_t tP = tS;  // P (bf16) overwrites the first half of S
 #pragma unroll
       for (int k = 0; k < kBlockN / 32; ++k) {
@@ -251,18 +253,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int c0 = 32 * k + 2 * i;
-          const float e0 = ex2_approx(fmaf(s[c0], c, neg));
-          const float e1 = ex2_approx(fmaf(s[c0 + 1], c, neg));
-          sum[(2 * i) & 3] += e0;
-          sum[(2 * i + 1) & 3] += e1;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[c0], s[c0 + 1]), cc, nn), x0, x1);
+          const float e0 = ex2_approx(x0);
+          const float e1 = ex2_approx(x1);
+          acc[i & 3] = f2_add(acc[i & 3], f2_pack(e0, e1));
           pk[i] = pack_bf16x2(e0, e1);
         }
         tmem_st16(tP + 16 * k, pk);
       }
+      float sum[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) f2_unpack(acc[i], sum[2 * i], sum[2 * i + 1]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(BAR_P + t));
-      l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+      l = l * alpha + (((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7])));
       m_raw = mx;
       m_sc = m_sc_new;
     }
@@ -294,8 +300,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t r[32];
             tmem_ld32(tO + 32 * ch, r);
             tmem_wait_ld();
+            const uint64_t aa = f2_pack(alpha, alpha);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            for (int i = 0; i < 16; ++i) {
+              float lo, hi;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), aa), lo, hi);
+              r[2 * i] = __float_as_uint(lo);
+              r[2 * i + 1] = __float_as_uint(hi);
+            }
             tmem_st32(tO + 32 * ch, r);
           }
           tmem_wait_st();
@@ -352,8 +364,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (valid) p.lse[(static_cast<size_t>(b) * p.Hq + hq) * p.Nq + row] = lse;
     }
   } else if (warp == 12) {
-    // ========================= MMA issuer (one thread) =========================
-    if (lane == 0 && aligned_ok) {
+    // ============================ MMA issuer warp ============================
+    // The whole warp follows the schedule (warp-uniform waits and descriptor
+    // arithmetic); one elected lane -- always the same one in a converged warp,
+    // so its commits cover its own MMAs -- issues each group of tcgen05
+    // instructions (8 MMAs and their commit) inside a single elected block.
+    // Measured on B200: a group issued this way takes ~23 cycles per MMA and
+    // runs ahead of the tensor core, while a per-MMA elect/warp-sync costs
+    // 50-60 cycles each and a single divergent lane is slower still when the
+    // softmax warps sharing this SM sub-partition keep the issue slots busy.
+    if (aligned_ok) {
       const uint32_t idS = idesc_bf16_f32(kBlockM, kBlockN, false, p.negate != 0);
       const uint32_t idPV = idesc_bf16_f32(kBlockM, D, true, false);
       const uint32_t sQ = sbase + C::kOffQ;
@@ -366,111 +386,128 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dQ = sw128_desc(sQ, 16, 1024);             // K-major, 8-row groups 1 KiB apart
       const uint64_t dK = sw128_desc(sKV, 16, 1024);            // K-major
       const uint64_t dV = sw128_desc(sKV, kChunkBytes, 1024);   // MN-major: d-chunks 16 KiB apart
-      auto issue_s = [&](int t, int st) {
+      auto commit = [&](uint32_t b) {
+        if (elect_one()) umma_commit(b);
+        __syncwarp();
+      };
+      // S_t = Q_t K^T for the K tile in stage `st`, then commit to `c1` (and `c2`)
+      auto issue_s = [&](int t, int st, uint32_t c1, uint32_t c2) {
         const uint64_t a0 = dQ + ((t * C::kTileBytes) >> 4);
         const uint64_t b0 = dK + ((st * C::kTileBytes) >> 4);
+        const uint32_t dS = tmem + C::col_s(t);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
-          umma_ss(tmem + C::col_s(t), a0 + off, b0 + off, idS, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
+            umma_ss(dS, a0 + off, b0 + off, idS, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(c1);
+          if (c2) umma_commit(c2);
         }
+        __syncwarp();
       };
-      auto issue_pv = [&](int t, int st, bool acc) {
+      // O_t += P_t V for the V tile in stage `st`, then commit to `c1` (and `c2`)
+      auto issue_pv = [&](int t, int st, bool acc, uint32_t c1, uint32_t c2) {
         const uint64_t b0 = dV + ((st * C::kTileBytes) >> 4);
+        const uint32_t dO = tmem + C::col_o(t), aP = tmem + C::col_s(t);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          umma_ts(tmem + C::col_o(t), tmem + C::col_s(t) + kk * 8,
-                  b0 + ((kk * 16 * kSwizzleBytes) >> 4), idPV, (acc || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kBlockN / 16; ++kk)
+            umma_ts(dO, aP + kk * 8, b0 + ((kk * 16 * kSwizzleBytes) >> 4), idPV,
+                    (acc || kk > 0) ? 1u : 0u);
+          if (c1) umma_commit(c1);
+          if (c2) umma_commit(c2);
         }
+        __syncwarp();
       };
       bool ok = true;
-      for (int t = 0; t < 2 && ok; ++t)
-        if ((t ? nt1 : nt0) > 0) ok = mbar_wait(bar(BAR_Q + t), 0, g, FA2_SITE_Q_LOADED, t);
+      if (nt0 > 0) ok = mbar_wait_warp(bar(BAR_Q + 0), 0, g, FA2_SITE_Q_LOADED, 0);
+      if (ok && nt1 > 0) ok = mbar_wait_warp(bar(BAR_Q + 1), 0, g, FA2_SITE_Q_LOADED, 1);
       if (ok && n_kv > 0) {
-        ok = mbar_wait(bar(BAR_KV_FULL + stage_of(0)), phase_of(0), g, FA2_SITE_KV_LOADED, 0);
+        ok = mbar_wait_warp(bar(BAR_KV_FULL + stage_of(0)), phase_of(0), g, FA2_SITE_KV_LOADED, 0);
         if (ok) {
           tc_fence_after();
-          for (int t = 0; t < 2; ++t)
-            if ((t ? nt1 : nt0) > 0) {
-              issue_s(t, stage_of(0));
-              umma_commit(bar(BAR_S + t));
-            }
-          umma_commit(bar(BAR_KV_FULL + C::kStages + stage_of(0)));
+          if (nt0 > 0) issue_s(0, stage_of(0), bar(BAR_S + 0), 0);
+          if (nt1 > 0) issue_s(1, stage_of(0), bar(BAR_S + 1), 0);
+          commit(bar(BAR_KV_FULL + C::kStages + stage_of(0)));
         }
       }
       for (int j = 0; j < n_kv && ok; ++j) {
         const int itV = 2 * j + 1, itK = 2 * j + 2;
-        if (!mbar_wait(bar(BAR_KV_FULL + stage_of(itV)), phase_of(itV), g, FA2_SITE_KV_LOADED, j)) break;
+        if (!mbar_wait_warp(bar(BAR_KV_FULL + stage_of(itV)), phase_of(itV), g, FA2_SITE_KV_LOADED, j)) break;
         tc_fence_after();
         const bool next = (j + 1 < n_kv);
         // tile 0: O0 += P0 V_j, then S0(j+1)
         if (j < nt0) {
-          if (!mbar_wait(bar(BAR_P + 0), j & 1, g, FA2_SITE_P_READY, j)) break;
-          if (j > 0 && !mbar_wait(bar(BAR_ORESC + 0), (j - 1) & 1, g, FA2_SITE_O_RESCALED, j)) break;
+          if (!mbar_wait_warp(bar(BAR_P + 0), j & 1, g, FA2_SITE_P_READY, j)) break;
+          if (j > 0 && !mbar_wait_warp(bar(BAR_ORESC + 0), (j - 1) & 1, g, FA2_SITE_O_RESCALED, j)) break;
           tc_fence_after();
-          issue_pv(0, stage_of(itV), j > 0);
-          if (j == nt0 - 1) umma_commit(bar(BAR_OFINAL + 0));
+          // if tile 1 has no PV on V_j, this is its last use
+          issue_pv(0, stage_of(itV), j > 0, j == nt0 - 1 ? bar(BAR_OFINAL + 0) : 0u,
+                   j >= nt1 ? bar(BAR_KV_FULL + C::kStages + stage_of(itV)) : 0u);
         }
         if (next) {
-          if (!mbar_wait(bar(BAR_KV_FULL + stage_of(itK)), phase_of(itK), g, FA2_SITE_KV_LOADED, j + 1)) break;
+          if (!mbar_wait_warp(bar(BAR_KV_FULL + stage_of(itK)), phase_of(itK), g, FA2_SITE_KV_LOADED, j + 1)) break;
           tc_fence_after();
         }
-        if (j + 1 < nt0) {
-          issue_s(0, stage_of(itK));
-          umma_commit(bar(BAR_S + 0));
-        }
+        if (j + 1 < nt0)  // last use of K_{j+1} if tile 1 does not need it
+          issue_s(0, stage_of(itK), bar(BAR_S + 0),
+                  j + 1 >= nt1 ? bar(BAR_KV_FULL + C::kStages + stage_of(itK)) : 0u);
         // tile 1: O1 += P1 V_j, then S1(j+1)
         if (j < nt1) {
-          if (!mbar_wait(bar(BAR_P + 1), j & 1, g, FA2_SITE_P_READY, j)) break;
-          if (j > 0 && !mbar_wait(bar(BAR_ORESC + 1), (j - 1) & 1, g, FA2_SITE_O_RESCALED, j)) break;
+          if (!mbar_wait_warp(bar(BAR_P + 1), j & 1, g, FA2_SITE_P_READY, j)) break;
+          if (j > 0 && !mbar_wait_warp(bar(BAR_ORESC + 1), (j - 1) & 1, g, FA2_SITE_O_RESCALED, j)) break;
           tc_fence_after();
-          issue_pv(1, stage_of(itV), j > 0);
-          if (j == nt1 - 1) umma_commit(bar(BAR_OFINAL + 1));
+          // V_j may be overwritten once this (the last) PV on it completes
+          issue_pv(1, stage_of(itV), j > 0, bar(BAR_KV_FULL + C::kStages + stage_of(itV)),
+                   j == nt1 - 1 ? bar(BAR_OFINAL + 1) : 0u);
         }
-        umma_commit(bar(BAR_KV_FULL + C::kStages + stage_of(itV)));  // V_j may be overwritten
-        if (j + 1 < nt1) {
-          issue_s(1, stage_of(itK));
-          umma_commit(bar(BAR_S + 1));
-        }
-        if (next) umma_commit(bar(BAR_KV_FULL + C::kStages + stage_of(itK)));  // K_{j+1}
+        if (j + 1 < nt1)  // K_{j+1} may be overwritten once S1(j+1) completes
+          issue_s(1, stage_of(itK), bar(BAR_S + 1), bar(BAR_KV_FULL + C::kStages + stage_of(itK)));
       }
       // drain: every MMA issued above has completed before TMEM is released
       // (not cut short by the abort flag: tensor-core work always finishes)
       volatile int no_abort = 0;
       const WaitGuard drain{&no_abort, &g_status, p.limit_ns};
-      umma_commit(bar(BAR_DONE));
-      mbar_wait(bar(BAR_DONE), 0, drain, FA2_SITE_MMA_DRAIN, 0);
+      commit(bar(BAR_DONE));
+      mbar_wait_warp(bar(BAR_DONE), 0, drain, FA2_SITE_MMA_DRAIN, 0);
     }
-    __syncwarp();
   } else if (warp == 13) {
-    // ========================= TMA producer (one thread) =========================
-    if (lane == 0 && aligned_ok) {
+    // ============================ TMA producer warp ============================
+    if (aligned_ok) {
       const uint32_t sQ = sbase + C::kOffQ;
       const uint32_t sKV = sbase + C::kOffKV;
+#pragma unroll 1
       for (int t = 0; t < 2; ++t) {
         if ((t ? nt1 : nt0) == 0) continue;
-        mbar_arrive_expect_tx(bar(BAR_Q + t), C::kTileBytes);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(BAR_Q + t), C::kTileBytes);
 #pragma unroll
-        for (int ch = 0; ch < C::kChunks; ++ch)
-          tma_load_4d(sQ + t * C::kTileBytes + ch * kChunkBytes, &tmQ, bar(BAR_Q + t), ch * 64, hq,
-                      row0 + t * kBlockM, b);
+          for (int ch = 0; ch < C::kChunks; ++ch)
+            tma_load_4d(sQ + t * C::kTileBytes + ch * kChunkBytes, &tmQ, bar(BAR_Q + t), ch * 64, hq,
+                        row0 + t * kBlockM, b);
+        }
+        __syncwarp();
       }
       int issued = 0;
       bool ok = true;
       for (int it = 0; it < 2 * n_kv; ++it) {
         const int st = it % C::kStages;
         if (it >= C::kStages &&
-            !mbar_wait(bar(BAR_KV_FULL + C::kStages + st), ((it / C::kStages) & 1) ^ 1, g,
-                       FA2_SITE_KV_FREE, it)) {
+            !mbar_wait_warp(bar(BAR_KV_FULL + C::kStages + st), ((it / C::kStages) & 1) ^ 1, g,
+                            FA2_SITE_KV_FREE, it)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(bar(BAR_KV_FULL + st), C::kTileBytes);
-        const CUtensorMap* map = (it & 1) ? &tmV : &tmK;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(BAR_KV_FULL + st), C::kTileBytes);
+          const CUtensorMap* map = (it & 1) ? &tmV : &tmK;
 #pragma unroll
-        for (int ch = 0; ch < C::kChunks; ++ch)
-          tma_load_4d(sKV + st * C::kTileBytes + ch * kChunkBytes, map, bar(BAR_KV_FULL + st), ch * 64,
-                      hk, (it >> 1) * kBlockN, b);
+          for (int ch = 0; ch < C::kChunks; ++ch)
+            tma_load_4d(sKV + st * C::kTileBytes + ch * kChunkBytes, map, bar(BAR_KV_FULL + st),
+                        ch * 64, hk, (it >> 1) * kBlockN, b);
+        }
+        __syncwarp();
         issued = it + 1;
       }
       if (!ok) {
@@ -478,13 +515,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         volatile int no_abort = 0;
         const WaitGuard drain{&no_abort, &g_status, p.limit_ns};
         for (int it = (issued > C::kStages ? issued - C::kStages : 0); it < issued; ++it)
-          mbar_wait(bar(BAR_KV_FULL + it % C::kStages), (it / C::kStages) & 1, drain,
-                    FA2_SITE_LOAD_DRAIN, it);
-        for (int t = 0; t < 2; ++t)
-          if ((t ? nt1 : nt0) > 0) mbar_wait(bar(BAR_Q + t), 0, drain, FA2_SITE_LOAD_DRAIN, t);
+          mbar_wait_warp(bar(BAR_KV_FULL + it % C::kStages), (it / C::kStages) & 1, drain,
+                         FA2_SITE_LOAD_DRAIN, it);
+        if (nt0 > 0) mbar_wait_warp(bar(BAR_Q + 0), 0, drain, FA2_SITE_LOAD_DRAIN, 0);
+        if (nt1 > 0) mbar_wait_warp(bar(BAR_Q + 1), 0, drain, FA2_SITE_LOAD_DRAIN, 1);
       }
     }
-    __syncwarp();
   }
 
   // ---- teardown: all TMEM traffic is finished before the columns are freed ----

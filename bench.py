@@ -221,6 +221,29 @@ def run_reference(args, w):
     return 0
 
 
+def rank_seed(w, rank: int) -> int:
+    """Seed of rank `rank`'s independent batch (weak scaling: every rank runs
+    the full workload on its own inputs)."""
+    return w.seed + rank
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks of the default
+    process group (identity when torch.distributed is not initialised)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(x) for x in values]
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def throughput_tflops(w, world: int, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank processes one workload per step."""
+    return world * w.flops() / (ms_per_step * 1e-3) / 1e12
+
+
 def workload_config(w, n_gpus):
     return {"workload": w.name, "description": w.description, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
             "Nq": w.Nq, "Nk": w.Nk, "d": w.d, "causal": w.causal,
@@ -246,7 +269,7 @@ def run_fa2(args, w):
 
     import exact_tiled_attention_29_b200 as fa2
 
-    q_h, k_h, v_h = make_qkv(w, seed=w.seed + rank)
+    q_h, k_h, v_h = make_qkv(w, seed=rank_seed(w, rank))
     q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
@@ -295,10 +318,7 @@ def run_fa2(args, w):
     if dstat != 0:
         raise RuntimeError(f"device status {dstat:#x} after the timed region")
 
-    if world > 1:
-        t = torch.tensor([mean_ms, bracket_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        mean_ms, bracket_ms = float(t[0]), float(t[1])
+    mean_ms, bracket_ms = max_over_ranks([mean_ms, bracket_ms], device=dev)
 
     # ---- end-to-end through the public API with host buffers ----
     e2e = None
@@ -333,20 +353,16 @@ def run_fa2(args, w):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1) / n_e2e
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t[0])
+        e_ms = max_over_ranks([e0.elapsed_time(e1) / n_e2e], device=dev)[0]
         if not torch.isfinite(lp).any():
             raise RuntimeError("e2e produced no finite LSE")
         h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
         d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
-        e2e = {"value": world * w.flops() / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": throughput_tflops(w, world, e_ms), "unit": "TFLOP/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": n_e2e}
 
-    value = world * w.flops() / (mean_ms * 1e-3) / 1e12
+    value = throughput_tflops(w, world, mean_ms)
     line = None
     if rank == 0:
         peaks, peak_src = load_peaks()

@@ -32,6 +32,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/fa2.h"
 #include "sm100_ptx.cuh"
@@ -48,10 +49,10 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kSwizzleBytes = 128;  // one swizzle atom row: 64 bf16
 constexpr int kChunkBytes = kBlockM * kSwizzleBytes;  // 64 columns of a 128-row tile
 
-// Register split (per thread): 2 softmax warpgroups x 184 + correction 64 +
+// Register split (per thread): 2 softmax warpgroups x 192 + correction 48 +
 // MMA/load warpgroup 80 = 512 = 4 x 128, i.e. exactly the launch pool.
-constexpr int kRegsSoftmax = 184;
-constexpr int kRegsCorrection = 64;
+constexpr int kRegsSoftmax = 192;
+constexpr int kRegsCorrection = 48;
 constexpr int kRegsOther = 80;
 static_assert(2 * kRegsSoftmax + kRegsCorrection + kRegsOther == 4 * kLaunchRegs,
               "register split must equal the launch allocation");
@@ -59,13 +60,12 @@ static_assert(2 * kRegsSoftmax + kRegsCorrection + kRegsOther == 4 * kLaunchRegs
 enum Bar {
   BAR_Q = 0,         // [2] Q tile loaded (TMA tx)
   BAR_S = 2,         // [2] S tile complete (MMA commit)
-  BAR_P = 4,         // [2] P written to TMEM (128 softmax threads)
+  BAR_P = 4,         // [2] P written to TMEM and O rescaled (128 softmax + 128 correction threads)
   BAR_STATS = 6,     // [2] per-row rescale factor published (128 softmax threads)
-  BAR_ORESC = 8,     // [2] O rescaled (128 correction threads)
-  BAR_OFINAL = 10,   // [2] last PV complete (MMA commit)
-  BAR_FSTATS = 12,   // [2] final row max / denominator published
-  BAR_DONE = 14,     // all MMAs drained (MMA commit)
-  BAR_KV_FULL = 15,  // [stages]
+  BAR_OFINAL = 8,    // [2] last PV complete (MMA commit)
+  BAR_FSTATS = 10,   // [2] final row max / denominator published
+  BAR_DONE = 12,     // all MMAs drained (MMA commit)
+  BAR_KV_FULL = 13,  // [stages] K/V tile landed (TMA tx); then [stages] slot free (MMA commit)
 };
 
 template <int D>
@@ -115,6 +115,44 @@ __device__ __forceinline__ int kv_tiles_for(const Params& p, int r0) {
   return min(nkt, (int)(lim / kBlockN) + 1);
 }
 
+// 2^x for a pair of fp32 values on the FMA pipe instead of the MUFU: a
+// Cody-Waite split x = j + f with j = round(x), f in [-1/2, 1/2], then
+// 2^f ~= c0 + f(c1 + f(c2 + f c3)) and 2^j applied by adding j to the exponent
+// field.  The coefficients minimise the maximum relative error of the cubic on
+// [-1/2, 1/2] (Remez exchange, fitted for this kernel): 7.5e-5, far below the
+// 2^-9 rounding of the bf16 P it feeds.  Inputs are clamped at -125 so the
+// result stays a normal number (2^-125 ~ 2e-38 stands in for anything
+// smaller); callers use it only where no score is masked to -inf.
+constexpr float kExp2C0 = 9.999280572e-01f;
+constexpr float kExp2C1 = 6.932609677e-01f;
+constexpr float kExp2C2 = 2.426111251e-01f;
+constexpr float kExp2C3 = 5.517166853e-02f;
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& e0, float& e1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = f2_add(x, f2_pack(kRound, kRound));         // low mantissa bits hold j
+  const uint64_t jf = f2_add(t, f2_pack(-kRound, -kRound));      // j as a float
+  const uint64_t f = f2_fma(jf, f2_pack(-1.f, -1.f), x);         // f = x - j
+  uint64_t q = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+  q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
+  q = f2_fma(q, f, f2_pack(kExp2C0, kExp2C0));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  e0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  e1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
+// Pairs of each 32-column chunk whose exponentials go through exp2_poly_pair
+// in unmasked tiles (the rest use the MUFU).  It moves work from the MUFU to
+// the FMA pipe; measured on B200 it does not pay while the per-tile chain,
+// not MUFU throughput, bounds the kernel (2 or 4 pairs: -4 to -8 % on causal
+// 8k), so the default is 0.
+#ifndef FA2_EMU_PAIRS
+#define FA2_EMU_PAIRS 0
+#endif
+constexpr int kEmuPairs = FA2_EMU_PAIRS;
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -153,9 +191,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     for (int i = 0; i < BAR_KV_FULL; ++i) {
       uint32_t cnt = 1;
-      if ((i >= BAR_P && i < BAR_P + 2) || (i >= BAR_STATS && i < BAR_STATS + 2) ||
-          (i >= BAR_ORESC && i < BAR_ORESC + 2) || (i >= BAR_FSTATS && i < BAR_FSTATS + 2))
+      if ((i >= BAR_STATS && i < BAR_STATS + 2) || (i >= BAR_FSTATS && i < BAR_FSTATS + 2))
         cnt = kBlockM;
+      if (i >= BAR_P && i < BAR_P + 2) cnt = 2 * kBlockM;
       mbar_init(bar(i), cnt);
     }
     for (int s = 0; s < 2 * C::kStages; ++s) mbar_init(bar(BAR_KV_FULL + s), 1);
@@ -247,21 +285,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t cc = f2_pack(c, c), nn = f2_pack(-m_sc_new, -m_sc_new);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // packed partial row sums (+0.0f pairs)
       const uint32_t tP = tS;  // P (bf16) overwrites the first half of S
+      auto exp_row = [&](auto emu_tag) {
+        constexpr int kEmu = decltype(emu_tag)::value;
 #pragma unroll
-      for (int k = 0; k < kBlockN / 32; ++k) {
-        uint32_t pk[16];
+        for (int k = 0; k < kBlockN / 32; ++k) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c0 = 32 * k + 2 * i;
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s[c0], s[c0 + 1]), cc, nn), x0, x1);
-          const float e0 = ex2_approx(x0);
-          const float e1 = ex2_approx(x1);
-          acc[i & 3] = f2_add(acc[i & 3], f2_pack(e0, e1));
-          pk[i] = pack_bf16x2(e0, e1);
+          for (int i = 0; i < 16; ++i) {
+            const int c0 = 32 * k + 2 * i;
+            float x0, x1, e0, e1;
+            f2_unpack(f2_fma(f2_pack(s[c0], s[c0 + 1]), cc, nn), x0, x1);
+            if (i >= 16 - kEmu) {
+              exp2_poly_pair(x0, x1, e0, e1);
+            } else {
+              e0 = ex2_approx(x0);
+              e1 = ex2_approx(x1);
+            }
+            acc[i & 3] = f2_add(acc[i & 3], f2_pack(e0, e1));
+            pk[i] = pack_bf16x2(e0, e1);
+          }
+          tmem_st16(tP + 16 * k, pk);
         }
-        tmem_st16(tP + 16 * k, pk);
-      }
+      };
+      if (masked)  // masked scores are -inf and must give exactly 0: MUFU only
+        exp_row(std::integral_constant<int, 0>{});
+      else
+        exp_row(std::integral_constant<int, kEmuPairs>{});
       float sum[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) f2_unpack(acc[i], sum[2 * i], sum[2 * i + 1]);
@@ -281,10 +330,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rt = q4 * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     bool ok = true;
-    for (int j = 1; j < n_kv && ok; ++j) {
+    for (int j = 0; j < n_kv && ok; ++j) {
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if (j >= (t ? nt1 : nt0)) continue;
+        if (j == 0) {  // nothing accumulated yet: O_t is ready for the first PV
+          mbar_arrive(bar(BAR_P + t));
+          continue;
+        }
         if (!mbar_wait(bar(BAR_STATS + t), (j - 1) & 1, g, FA2_SITE_STATS_READY, j)) {
           ok = false;
           break;
@@ -295,25 +348,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           // softmax threads waited for before publishing alpha
           tc_fence_after();
           const uint32_t tO = tmem + lane_off + C::col_o(t);
+          const uint64_t aa = f2_pack(alpha, alpha);
 #pragma unroll 1
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t r[32];
-            tmem_ld32(tO + 32 * ch, r);
+          for (int ch = 0; ch < D / 16; ++ch) {
+            uint32_t r[16];
+            tmem_ld16(tO + 16 * ch, r);
             tmem_wait_ld();
-            const uint64_t aa = f2_pack(alpha, alpha);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
+            for (int i = 0; i < 8; ++i) {
               float lo, hi;
               f2_unpack(f2_mul(f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), aa), lo, hi);
               r[2 * i] = __float_as_uint(lo);
               r[2 * i + 1] = __float_as_uint(hi);
             }
-            tmem_st32(tO + 32 * ch, r);
+            tmem_st16(tO + 16 * ch, r);
           }
           tmem_wait_st();
         }
         tc_fence_before();
-        mbar_arrive(bar(BAR_ORESC + t));
+        mbar_arrive(bar(BAR_P + t));
       }
     }
     // epilogue: O / l -> bf16, LSE = ln(sum exp(scale * s))
@@ -341,24 +394,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Nq + row) * p.Hq + hq) * D;
       const uint32_t tO = tmem + lane_off + C::col_o(t);
 #pragma unroll 1
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t r[32];
+      for (int ch = 0; ch < D / 16; ++ch) {
+        uint32_t r[16];
         if (have_o) {
-          tmem_ld32(tO + 32 * ch, r);
+          tmem_ld16(tO + 16 * ch, r);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = 0u;
+          for (int i = 0; i < 16; ++i) r[i] = 0u;
         }
-        uint4 w[4];
+        uint4 w[2];
         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
+        for (int i = 0; i < 8; ++i)
           wp[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * ch);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = w[i];
+          uint4* dst = reinterpret_cast<uint4*>(orow + 16 * ch);
+          dst[0] = w[0];
+          dst[1] = w[1];
         }
       }
       if (valid) p.lse[(static_cast<size_t>(b) * p.Hq + hq) * p.Nq + row] = lse;
@@ -390,36 +443,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (elect_one()) umma_commit(b);
         __syncwarp();
       };
-      // S_t = Q_t K^T for the K tile in stage `st`, then commit to `c1` (and `c2`)
-      auto issue_s = [&](int t, int st, uint32_t c1, uint32_t c2) {
+      // One elected block per tile and KV step: O_t += P_t V_j, then (if any)
+      // S_t(j+1) = Q_t K_{j+1}^T, then the commits that publish completion.
+      // S_t(j+1) overwrites the TMEM columns that held P_t(j); it is issued by
+      // the same thread after the PV that reads them, and one thread's tcgen05
+      // MMAs execute in issue order.
+      auto issue_block = [&](int t, int j, bool pv, bool s_next, uint32_t c_pv1, uint32_t c_pv2,
+                             uint32_t c_s1, uint32_t c_s2) {
+        const uint32_t dS = tmem + C::col_s(t), dO = tmem + C::col_o(t);
+        const uint64_t bV = dV + ((stage_of(2 * j + 1) * C::kTileBytes) >> 4);
         const uint64_t a0 = dQ + ((t * C::kTileBytes) >> 4);
-        const uint64_t b0 = dK + ((st * C::kTileBytes) >> 4);
+        const uint64_t bK = dK + ((stage_of(2 * j + 2) * C::kTileBytes) >> 4);
+        if (elect_one()) {
+          if (pv) {
+#pragma unroll
+            for (int kk = 0; kk < kBlockN / 16; ++kk)
+              umma_ts(dO, dS + kk * 8, bV + ((kk * 16 * kSwizzleBytes) >> 4), idPV,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+            if (c_pv1) umma_commit(c_pv1);
+            if (c_pv2) umma_commit(c_pv2);
+          }
+          if (s_next) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
+              umma_ss(dS, a0 + off, bK + off, idS, kk > 0 ? 1u : 0u);
+            }
+            if (c_s1) umma_commit(c_s1);
+            if (c_s2) umma_commit(c_s2);
+          }
+        }
+        __syncwarp();
+      };
+      // S_t(0)
+      auto issue_s0 = [&](int t, uint32_t c2) {
         const uint32_t dS = tmem + C::col_s(t);
+        const uint64_t a0 = dQ + ((t * C::kTileBytes) >> 4);
+        const uint64_t bK = dK + ((stage_of(0) * C::kTileBytes) >> 4);
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
-            umma_ss(dS, a0 + off, b0 + off, idS, kk > 0 ? 1u : 0u);
+            umma_ss(dS, a0 + off, bK + off, idS, kk > 0 ? 1u : 0u);
           }
-          umma_commit(c1);
+          umma_commit(bar(BAR_S + t));
           if (c2) umma_commit(c2);
         }
         __syncwarp();
       };
-      // O_t += P_t V for the V tile in stage `st`, then commit to `c1` (and `c2`)
-      auto issue_pv = [&](int t, int st, bool acc, uint32_t c1, uint32_t c2) {
-        const uint64_t b0 = dV + ((st * C::kTileBytes) >> 4);
-        const uint32_t dO = tmem + C::col_o(t), aP = tmem + C::col_s(t);
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < kBlockN / 16; ++kk)
-            umma_ts(dO, aP + kk * 8, b0 + ((kk * 16 * kSwizzleBytes) >> 4), idPV,
-                    (acc || kk > 0) ? 1u : 0u);
-          if (c1) umma_commit(c1);
-          if (c2) umma_commit(c2);
-        }
-        __syncwarp();
-      };
+      auto free_of = [&](int it) { return bar(BAR_KV_FULL + C::kStages + stage_of(it)); };
       bool ok = true;
       if (nt0 > 0) ok = mbar_wait_warp(bar(BAR_Q + 0), 0, g, FA2_SITE_Q_LOADED, 0);
       if (ok && nt1 > 0) ok = mbar_wait_warp(bar(BAR_Q + 1), 0, g, FA2_SITE_Q_LOADED, 1);
@@ -427,43 +499,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait_warp(bar(BAR_KV_FULL + stage_of(0)), phase_of(0), g, FA2_SITE_KV_LOADED, 0);
         if (ok) {
           tc_fence_after();
-          if (nt0 > 0) issue_s(0, stage_of(0), bar(BAR_S + 0), 0);
-          if (nt1 > 0) issue_s(1, stage_of(0), bar(BAR_S + 1), 0);
-          commit(bar(BAR_KV_FULL + C::kStages + stage_of(0)));
+          if (nt0 > 0) issue_s0(0, nt1 > 0 ? 0u : free_of(0));
+          if (nt1 > 0) issue_s0(1, free_of(0));
         }
       }
       for (int j = 0; j < n_kv && ok; ++j) {
         const int itV = 2 * j + 1, itK = 2 * j + 2;
-        if (!mbar_wait_warp(bar(BAR_KV_FULL + stage_of(itV)), phase_of(itV), g, FA2_SITE_KV_LOADED, j)) break;
-        tc_fence_after();
         const bool next = (j + 1 < n_kv);
-        // tile 0: O0 += P0 V_j, then S0(j+1)
+        // operands of this step (normally landed long ago); checked while the
+        // tensor pipe still holds the previous block
+        if (!mbar_wait_warp(bar(BAR_KV_FULL + stage_of(itV)), phase_of(itV), g, FA2_SITE_KV_LOADED, j)) break;
+        if (next && !mbar_wait_warp(bar(BAR_KV_FULL + stage_of(itK)), phase_of(itK), g,
+                                    FA2_SITE_KV_LOADED, j + 1))
+          break;
+        // tile 0: PV0(j) and S0(j+1); V_j / K_{j+1} are freed here when tile 1 has no use for them
         if (j < nt0) {
           if (!mbar_wait_warp(bar(BAR_P + 0), j & 1, g, FA2_SITE_P_READY, j)) break;
-          if (j > 0 && !mbar_wait_warp(bar(BAR_ORESC + 0), (j - 1) & 1, g, FA2_SITE_O_RESCALED, j)) break;
           tc_fence_after();
-          // if tile 1 has no PV on V_j, this is its last use
-          issue_pv(0, stage_of(itV), j > 0, j == nt0 - 1 ? bar(BAR_OFINAL + 0) : 0u,
-                   j >= nt1 ? bar(BAR_KV_FULL + C::kStages + stage_of(itV)) : 0u);
+          issue_block(0, j, true, j + 1 < nt0, j == nt0 - 1 ? bar(BAR_OFINAL + 0) : 0u,
+                      j >= nt1 ? free_of(itV) : 0u, bar(BAR_S + 0), j + 1 >= nt1 ? free_of(itK) : 0u);
         }
-        if (next) {
-          if (!mbar_wait_warp(bar(BAR_KV_FULL + stage_of(itK)), phase_of(itK), g, FA2_SITE_KV_LOADED, j + 1)) break;
-          tc_fence_after();
-        }
-        if (j + 1 < nt0)  // last use of K_{j+1} if tile 1 does not need it
-          issue_s(0, stage_of(itK), bar(BAR_S + 0),
-                  j + 1 >= nt1 ? bar(BAR_KV_FULL + C::kStages + stage_of(itK)) : 0u);
-        // tile 1: O1 += P1 V_j, then S1(j+1)
+        // tile 1: PV1(j) and S1(j+1); the last use of V_j and K_{j+1}
         if (j < nt1) {
           if (!mbar_wait_warp(bar(BAR_P + 1), j & 1, g, FA2_SITE_P_READY, j)) break;
-          if (j > 0 && !mbar_wait_warp(bar(BAR_ORESC + 1), (j - 1) & 1, g, FA2_SITE_O_RESCALED, j)) break;
           tc_fence_after();
-          // V_j may be overwritten once this (the last) PV on it completes
-          issue_pv(1, stage_of(itV), j > 0, bar(BAR_KV_FULL + C::kStages + stage_of(itV)),
-                   j == nt1 - 1 ? bar(BAR_OFINAL + 1) : 0u);
+          issue_block(1, j, true, j + 1 < nt1, free_of(itV), j == nt1 - 1 ? bar(BAR_OFINAL + 1) : 0u,
+                      bar(BAR_S + 1), free_of(itK));
         }
-        if (j + 1 < nt1)  // K_{j+1} may be overwritten once S1(j+1) completes
-          issue_s(1, stage_of(itK), bar(BAR_S + 1), bar(BAR_KV_FULL + C::kStages + stage_of(itK)));
       }
       // drain: every MMA issued above has completed before TMEM is released
       // (not cut short by the abort flag: tensor-core work always finishes)

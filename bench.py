@@ -52,6 +52,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--schedule", default="streamk", choices=["streamk", "units"],
+                    help="streamk: fa2_forward_ws, one persistent block per SM over a workspace; "
+                         "units: fa2_forward, one block per (query block, head, batch)")
     return ap.parse_args()
 
 
@@ -213,7 +216,7 @@ def run_reference(args, w):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(w, args.gpus),
+            "config": workload_config(w, args.gpus, args.schedule),
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": orc.default_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -244,8 +247,8 @@ def throughput_tflops(w, world: int, ms_per_step: float) -> float:
     return world * w.flops() / (ms_per_step * 1e-3) / 1e12
 
 
-def workload_config(w, n_gpus):
-    return {"workload": w.name, "description": w.description, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+def workload_config(w, n_gpus, schedule="streamk"):
+    return {"workload": w.name, "schedule": schedule, "description": w.description, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
             "Nq": w.Nq, "Nk": w.Nk, "d": w.d, "causal": w.causal,
             "softmax_scale": w.softmax_scale, "seed": w.seed,
             "flops_per_step_per_rank": w.flops(),
@@ -276,11 +279,23 @@ def run_fa2(args, w):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def forward():
-        st = fa2.fa2_forward(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
-                             w.softmax_scale, stream)
+    # stream-K needs a zero-filled workspace once; calls ordered on one stream reuse it
+    ws = None
+    if args.schedule == "streamk":
+        ws = fa2.alloc_workspace(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal, dev)
+
+    def call(qq, kk, vv, oo, ll):
+        if ws is None:
+            st = fa2.fa2_forward(qq, kk, vv, oo, ll, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
+                                 w.softmax_scale, stream)
+        else:
+            st = fa2.fa2_forward_ws(qq, kk, vv, oo, ll, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d,
+                                    w.causal, w.softmax_scale, ws, ws.numel(), stream)
         if st != 0:
             raise fa2.FA2Error(st)
+
+    def forward():
+        call(q, k, v, o, lse)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -334,10 +349,7 @@ def run_fa2(args, w):
             qd.copy_(qp, non_blocking=True)
             kd.copy_(kp, non_blocking=True)
             vd.copy_(vp, non_blocking=True)
-            st = fa2.fa2_forward(qd, kd, vd, od, ld, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
-                                 w.softmax_scale, stream)
-            if st != 0:
-                raise fa2.FA2Error(st)
+            call(qd, kd, vd, od, ld)
             op.copy_(od, non_blocking=True)
             lp.copy_(ld, non_blocking=True)
 
@@ -377,7 +389,7 @@ def run_fa2(args, w):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(w, world),
+            "config": workload_config(w, world, args.schedule),
             "pct_of_peak": 100.0 * achieved / peak,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,

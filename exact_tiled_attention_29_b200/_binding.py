@@ -18,12 +18,12 @@ FA2_OK = 0
 STATUS_NAMES = {
     0: "FA2_OK", 1: "FA2_ERR_NULL_POINTER", 2: "FA2_ERR_BAD_SHAPE", 3: "FA2_ERR_HEAD_DIM",
     4: "FA2_ERR_ALIGNMENT", 5: "FA2_ERR_SCALE", 6: "FA2_ERR_DEVICE", 7: "FA2_ERR_LAUNCH",
-    8: "FA2_ERR_SIZE", 9: "FA2_ERR_BUILD",
+    8: "FA2_ERR_SIZE", 9: "FA2_ERR_BUILD", 10: "FA2_ERR_WORKSPACE",
 }
 SITE_NAMES = {
     1: "Q_LOADED", 2: "KV_LOADED", 3: "KV_FREE", 4: "S_READY", 5: "P_READY", 6: "STATS_READY",
     7: "O_RESCALED", 8: "O_FINAL", 9: "FINAL_STATS", 10: "MMA_DRAIN", 11: "LOAD_DRAIN",
-    15: "SELFTEST",
+    12: "MERGE", 15: "SELFTEST",
 }
 FA2_SITE_SELFTEST = 15
 
@@ -42,6 +42,10 @@ def _load() -> ctypes.CDLL:
     vp, ci, cf, cll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
     lib.fa2_forward.argtypes = [vp, vp, vp, vp, vp] + [ci] * 7 + [cf, vp]
     lib.fa2_forward.restype = ci
+    lib.fa2_forward_ws.argtypes = [vp, vp, vp, vp, vp] + [ci] * 7 + [cf, vp, cll, vp]
+    lib.fa2_forward_ws.restype = ci
+    lib.fa2_workspace_size.argtypes = [ci] * 7
+    lib.fa2_workspace_size.restype = cll
     lib.fa2_status_string.argtypes = [ci]
     lib.fa2_status_string.restype = ctypes.c_char_p
     lib.fa2_debug_status.argtypes = [vp]
@@ -53,6 +57,9 @@ def _load() -> ctypes.CDLL:
     ip = ctypes.POINTER(ci)
     lib.fa2_launch_plan.argtypes = [ci] * 6 + [ip] * 4
     lib.fa2_launch_plan.restype = ci
+    llp = ctypes.POINTER(cll)
+    lib.fa2_streamk_plan.argtypes = [ci] * 8 + [llp, ip, llp]
+    lib.fa2_streamk_plan.restype = ci
     return lib
 
 
@@ -84,6 +91,29 @@ def fa2_forward(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, s
                                 float(softmax_scale), _stream(stream)))
 
 
+def fa2_forward_ws(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, workspace,
+                   workspace_bytes, stream) -> int:
+    """Stream-K variant over a caller-provided workspace.  Returns the status code."""
+    return int(_lib.fa2_forward_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(Hq),
+                                   int(Hkv), int(Nq), int(Nk), int(d), int(bool(causal)),
+                                   float(softmax_scale), _ptr(workspace), int(workspace_bytes),
+                                   _stream(stream)))
+
+
+def fa2_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal) -> int:
+    return int(_lib.fa2_workspace_size(int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
+                                       int(bool(causal))))
+
+
+def fa2_streamk_plan(B, Hq, Hkv, Nq, Nk, d, causal, num_sms):
+    """(status, total_iters, ctas, workspace_bytes)."""
+    t, g, w = ctypes.c_longlong(0), ctypes.c_int(0), ctypes.c_longlong(0)
+    st = _lib.fa2_streamk_plan(int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
+                               int(bool(causal)), int(num_sms), ctypes.byref(t), ctypes.byref(g),
+                               ctypes.byref(w))
+    return int(st), t.value, g.value, w.value
+
+
 def fa2_status_string(status: int) -> str:
     return _lib.fa2_status_string(int(status)).decode()
 
@@ -110,12 +140,28 @@ def fa2_launch_plan(B, Hq, Hkv, Nq, Nk, d):
 
 # ---- torch convenience: allocate outputs with torch, then call the C ABI ----
 
+def alloc_workspace(B, Hq, Hkv, Nq, Nk, d, causal, device):
+    """A zero-filled uint8 CUDA tensor large enough for ``fa2_forward_ws``.
+
+    Zero once here; every completed call leaves the counters zero again, so
+    the tensor can be reused by later calls ordered on the same stream.
+    """
+    import torch
+
+    n = fa2_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal)
+    if n < 0:
+        raise FA2Error(2, "fa2_workspace_size")
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
+
+
 def attention(q, k, v, causal: bool = False, softmax_scale: float | None = None, out=None,
-              lse=None, stream=None):
+              lse=None, stream=None, workspace=None):
     """O, LSE for bf16 CUDA tensors q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d] (contiguous).
 
     Outputs are allocated with torch unless given; the work is one call to
-    ``fa2_forward`` on ``stream`` (default: torch's current stream).
+    ``fa2_forward`` on ``stream`` (default: torch's current stream), or to
+    ``fa2_forward_ws`` (stream-K schedule) when ``workspace`` -- a CUDA tensor
+    from ``alloc_workspace`` -- is given.
     """
     import torch
 
@@ -134,7 +180,13 @@ def attention(q, k, v, causal: bool = False, softmax_scale: float | None = None,
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    st = fa2_forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, stream)
+    if workspace is None:
+        st = fa2_forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, stream)
+        where = "fa2_forward"
+    else:
+        st = fa2_forward_ws(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale,
+                            workspace, workspace.numel() * workspace.element_size(), stream)
+        where = "fa2_forward_ws"
     if st != FA2_OK:
-        raise FA2Error(st)
+        raise FA2Error(st, where)
     return out, lse

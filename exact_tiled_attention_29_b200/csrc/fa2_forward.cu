@@ -49,24 +49,40 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kSwizzleBytes = 128;  // one swizzle atom row: 64 bf16
 constexpr int kChunkBytes = kBlockM * kSwizzleBytes;  // 64 columns of a 128-row tile
 
-// Register split (per thread): 2 softmax warpgroups x 192 + correction 48 +
-// MMA/load warpgroup 80 = 512 = 4 x 128, i.e. exactly the launch pool.
-constexpr int kRegsSoftmax = 192;
-constexpr int kRegsCorrection = 48;
+// Register split (per thread): 2 softmax warpgroups x 184 + correction/epilogue
+// 64 + MMA/load warpgroup 80 = 512 = 4 x 128, i.e. exactly the launch pool.
+// Each role compiles without spills in its budget.
+constexpr int kRegsSoftmax = 184;
+constexpr int kRegsCorrection = 64;
 constexpr int kRegsOther = 80;
 static_assert(2 * kRegsSoftmax + kRegsCorrection + kRegsOther == 4 * kLaunchRegs,
               "register split must equal the launch allocation");
 
 enum Bar {
-  BAR_Q = 0,         // [2] Q tile loaded (TMA tx)
+  BAR_Q = 0,         // Q tiles of the current piece loaded (TMA tx)
+  BAR_QFREE = 1,     // the current piece's last S MMA completed: Q smem reusable (MMA commit)
   BAR_S = 2,         // [2] S tile complete (MMA commit)
   BAR_P = 4,         // [2] P written to TMEM and O rescaled (128 softmax + 128 correction threads)
   BAR_STATS = 6,     // [2] per-row rescale factor published (128 softmax threads)
-  BAR_OFINAL = 8,    // [2] last PV complete (MMA commit)
-  BAR_FSTATS = 10,   // [2] final row max / denominator published
-  BAR_DONE = 12,     // all MMAs drained (MMA commit)
-  BAR_KV_FULL = 13,  // [stages] K/V tile landed (TMA tx); then [stages] slot free (MMA commit)
+  BAR_OFINAL = 8,    // [2] last PV of a piece complete (MMA commit)
+  BAR_FSTATS = 10,   // [2] final row max / denominator of a piece published (128 softmax threads)
+  BAR_FCONS = 12,    // [2] final statistics read by the epilogue (128 correction threads)
+  BAR_DONE = 14,     // all MMAs drained (MMA commit)
+  BAR_GRP = 15,      // a split piece's partial is fully published (128 correction threads)
+  BAR_MJOB = 16,     // merge job posted for a split piece (one correction thread)
+  BAR_MFREE = 17,    // merge job slot read (64 merge threads)
+  BAR_KV_FULL = 18,  // [stages] K/V tile landed (TMA tx); then [stages] slot free (MMA commit)
 };
+
+// Scheduling cost of a unit, in K/V-tile iterations, on top of its
+// iterations: the pipeline fill (Q load, first S) and the epilogue a unit
+// pays however short it is.  Stream-K cuts the summed costs into equal
+// ranges, so SMs that get many short units (the tail of a causal order) get
+// fewer iterations.
+constexpr int kUnitCost = 2;
+
+// Warps 14-15 (otherwise idle) merge split units and write empty ones.
+constexpr int kMergeThreads = 64;
 
 template <int D>
 struct Cfg {
@@ -86,6 +102,14 @@ struct Cfg {
   // TMEM column of S_t (P_t reuses its first half) and of O_t
   __host__ __device__ static constexpr uint32_t col_s(int t) { return t ? 128u : 0u; }
   __host__ __device__ static constexpr uint32_t col_o(int t) { return 256u + (t ? D : 0); }
+  // floats of one stream-K partial: O as [2 tiles][D/16 chunks][128 rows][16],
+  // then m [2][128] and l [2][128]
+  static constexpr int kPieceFloats = kTiles * kBlockM * (D + 2);
+  __host__ __device__ static constexpr int part_o(int t, int ch, int row) {
+    return ((t * (D / 16) + ch) * kBlockM + row) * 16;
+  }
+  __host__ __device__ static constexpr int part_m(int t, int row) { return kTiles * kBlockM * D + t * kBlockM + row; }
+  __host__ __device__ static constexpr int part_l(int t, int row) { return part_m(t, row) + kTiles * kBlockM; }
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(256 + 2 * D <= (int)kTmemCols, "TMEM budget");
 };
@@ -98,22 +122,217 @@ struct Params {
   int n_qblk;
   float c;            // |softmax_scale| * log2(e)
   int negate;         // softmax_scale < 0: compute S = -(Q K^T) so c stays >= 0
-  unsigned long long limit_ns;
+  uint32_t limit_ns;  // per bounded wait
+  // work decomposition
+  int streamk;        // 0: CTA i runs unit i whole; 1: CTA c runs cost positions [c*T/G, (c+1)*T/G)
+  int T;              // summed unit costs, kUnitCost + iterations per unit (< 2^31, checked on the host)
+  int span;           // T / G
+  int rem;            // T % G
+  int G;              // CTAs of a stream-K launch
+  float* ws;          // stream-K partials: [G CTAs][2: first / last piece of its range][piece floats]
+  int* ws_ctr;        // [G] arrival counters, zero before the launch and left zero after it
 };
 
-__device__ int g_status = 0;
-
-// Number of K/V tiles query tile t of this CTA visits (0 if it has no valid row
-// or no visible key).
-__device__ __forceinline__ int kv_tiles_for(const Params& p, int r0) {
-  if (r0 >= p.Nq) return 0;
-  const int nkt = (p.Nk + kBlockN - 1) / kBlockN;
-  if (!p.causal) return nkt;
-  const int rlast = min(r0 + kBlockM - 1, p.Nq - 1);
-  const long lim = (long)rlast + (long)p.Nk - (long)p.Nq;  // last visible key of the last row
+// Number of K/V tiles a 128-row query tile starting at row r0 visits (0 if it
+// has no valid row or no visible key).
+__host__ __device__ inline int kv_tiles_for(int Nq, int Nk, int causal, int r0) {
+  if (r0 >= Nq) return 0;
+  const int nkt = (Nk + kBlockN - 1) / kBlockN;
+  if (!causal) return nkt;
+  const int rlast = (r0 + kBlockM - 1 < Nq - 1) ? r0 + kBlockM - 1 : Nq - 1;
+  const long long lim = (long long)rlast + (long long)Nk - (long long)Nq;  // last visible key of the last row
   if (lim < 0) return 0;
-  return min(nkt, (int)(lim / kBlockN) + 1);
+  const long long t = lim / kBlockN + 1;
+  return t < nkt ? (int)t : nkt;
 }
+
+// K/V tiles of a unit (query block qb): the longer of its two query tiles.
+__host__ __device__ inline int unit_tiles(int Nq, int Nk, int causal, int qb) {
+  const int a = kv_tiles_for(Nq, Nk, causal, qb * kRowsPerCta);
+  const int b = kv_tiles_for(Nq, Nk, causal, qb * kRowsPerCta + kBlockM);
+  return a > b ? a : b;
+}
+
+// Start of CTA c's iteration range, floor(c * T / G), in 32-bit arithmetic:
+// c*T/G = c*span + c*rem/G with T = span*G + rem, c*span <= T < 2^31 and
+// c*rem < G*G.
+__host__ __device__ inline int range_start(int span, int rem, int G, int c) {
+  return c * span + (c * rem) / G;
+}
+
+// ---------------------------------------------------------------------------
+// Work decomposition, evaluated identically by every role of a CTA.
+//
+// Units are (256-row query block, query head, batch) in heaviest-first order:
+// round r holds the B*Hq units of query block n_qblk-1-r, (batch, head)
+// fastest; all units of a round need the same number of K/V tiles.  A piece
+// is a contiguous range [jb, je) of one unit's K/V tiles run by one CTA.
+//
+// Stream-K: the iterations of all units, concatenated in that order, are cut
+// into G equal ranges, one per CTA, so every SM gets the same number of
+// K/V-tile iterations (no wave quantisation, no long-unit tail).  A unit cut
+// by a range boundary is split; its pieces are merged through the workspace.
+// ---------------------------------------------------------------------------
+struct Piece {
+  int b, hq, qb;
+  int jb, je;       // K/V tiles [jb, je) of the unit
+  int nt0, nt1;     // K/V tiles of Q0 / Q1 over the whole unit
+  int a0, a1;       // iterations of Q0 / Q1 in this piece
+  int split;        // the unit is shared with other pieces
+  int slot;         // CTA that runs the unit's first piece (its counter is the unit's)
+  int npieces;      // pieces of the unit
+  int index;        // this piece's position in the unit
+};
+
+// Smallest c in [1, G] with B_c > y (G when no boundary lies above y): binary
+// search over the CTAs' range starts.
+__device__ __forceinline__ int first_boundary_above(const Params& p, int y) {
+  int lo = 1, hi = p.G;  // answer in [lo, hi]
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (range_start(p.span, p.rem, p.G, mid) > y) hi = mid; else lo = mid + 1;
+  }
+  return lo;
+}
+
+// Cost positions: round r's units are laid out one after another, unit k of
+// round r at [cum_r + k*w_r, cum_r + (k+1)*w_r) with w_r = kUnitCost + n_r
+// (0 for a round of empty units); iteration j of the unit sits at position
+// cum_r + k*w_r + kUnitCost + j.  CTA c runs the iterations whose positions
+// fall in [B_c, B_{c+1}), B_c = floor(c*T/G).
+//
+// Order of a CTA's pieces: when its range ends inside a unit that continues
+// on the next CTA, that piece (the unit's head) runs first and the rest in
+// order.  The next CTA starts with the same unit's tail, so both pieces of a
+// split unit finish early and its merge overlaps the remaining work instead
+// of landing at the end of the kernel.
+struct PieceIter {
+  int HB, r, n, k_cur;
+  int cum, x, x_end;  // cost before round r; the natural walk's range [x, x_end)
+  int state;          // unit mode: 1 = unit pending; stream-K: 1 = head piece pending
+
+  __device__ __forceinline__ static int cost(int n) { return n > 0 ? n + kUnitCost : 0; }
+
+  __device__ __forceinline__ void fill(const Params& p, Piece& pc, int r_, int k, int jb, int je) const {
+    pc.qb = p.n_qblk - 1 - r_;
+    pc.b = k / p.Hq;
+    pc.hq = k % p.Hq;
+    pc.jb = jb;
+    pc.je = je;
+    pc.nt0 = kv_tiles_for(p.Nq, p.Nk, p.causal, pc.qb * kRowsPerCta);
+    pc.nt1 = kv_tiles_for(p.Nq, p.Nk, p.causal, pc.qb * kRowsPerCta + kBlockM);
+    pc.a0 = max(0, min(je, pc.nt0) - jb);
+    pc.a1 = max(0, min(je, pc.nt1) - jb);
+  }
+
+  // (batch, head, query block) of the current piece, recomputed from the
+  // iterator so a role need not keep them live through its inner loop.
+  __device__ __forceinline__ void coords(const Params& p, Piece& pc) const {
+    pc.qb = p.n_qblk - 1 - r;
+    pc.b = k_cur / p.Hq;
+    pc.hq = k_cur % p.Hq;
+  }
+
+  // Which pieces share the current piece's unit: the range boundaries B_c
+  // (c = 1..G-1) that fall strictly inside the unit's iteration positions.
+  __device__ __forceinline__ void split_info(const Params& p, Piece& pc) const {
+    pc.split = 0;
+    pc.slot = 0;
+    pc.npieces = 1;
+    pc.index = 0;
+    if (!p.streamk) return;
+    const int s_u = cum + k_cur * cost(n) + kUnitCost;                // position of iteration 0
+    const int c_first = first_boundary_above(p, s_u);                // B_c > s_u
+    const int c_last = first_boundary_above(p, s_u + n - 1) - 1;     // B_c <= s_u + n - 1
+    if (c_last >= c_first) {
+      pc.split = 1;
+      pc.npieces = c_last - c_first + 2;
+      pc.slot = c_first - 1;
+      // pieces start at iteration 0 and at each inside boundary
+      const int ci = first_boundary_above(p, s_u + pc.jb) - 1;  // last boundary <= s_u + jb
+      pc.index = (ci < c_first) ? 0 : min(ci, c_last) - c_first + 1;
+    }
+  }
+
+  // Round state (r, cum, n) of the round holding cost position `pos`.
+  __device__ __forceinline__ void seek_round(const Params& p, int pos) {
+    r = 0;
+    cum = 0;
+    n = unit_tiles(p.Nq, p.Nk, p.causal, p.n_qblk - 1);
+    while (pos >= cum + HB * cost(n)) {  // the end of a round is at most T < 2^31
+      cum += HB * cost(n);
+      ++r;
+      n = unit_tiles(p.Nq, p.Nk, p.causal, p.n_qblk - 1 - r);
+    }
+  }
+
+  __device__ __forceinline__ void init(const Params& p) {
+    HB = p.B * p.Hq;
+    r = cum = n = k_cur = 0;
+    x = x_end = 0;
+    state = 1;
+    if (!p.streamk) return;
+    x = range_start(p.span, p.rem, p.G, blockIdx.x);
+    x_end = range_start(p.span, p.rem, p.G, blockIdx.x + 1);
+    state = 0;
+    if (x_end <= x) return;
+    // the unit holding the range's last position, and whether it continues
+    // past the range while the range also holds earlier units
+    seek_round(p, x_end - 1);
+    const int w = cost(n);
+    const int k = (x_end - 1 - cum) / w;
+    const int s_u = cum + k * w;
+    if (s_u > x && x_end - 1 >= s_u + kUnitCost && x_end < s_u + w) {
+      state = 1;
+      k_cur = k;
+      x_end = s_u;  // the natural walk stops where the head piece begins
+    }
+  }
+
+  __device__ __forceinline__ bool next(const Params& p, Piece& pc) {
+    if (!p.streamk) {
+      if (!state) return false;
+      state = 0;
+      const int u = blockIdx.x;
+      r = u / HB;
+      k_cur = u % HB;
+      const int nn = unit_tiles(p.Nq, p.Nk, p.causal, p.n_qblk - 1 - r);
+      if (nn == 0) return false;  // nothing to compute: the merge warps write this unit's empty rows
+      cum = 0;
+      n = nn;
+      fill(p, pc, r, k_cur, 0, nn);
+      return true;
+    }
+    if (state) {  // the head piece: iterations [0, B_{c+1} - position of iteration 0)
+      state = 0;
+      const int end = range_start(p.span, p.rem, p.G, blockIdx.x + 1);
+      fill(p, pc, r, k_cur, 0, end - (cum + k_cur * cost(n) + kUnitCost));
+      return true;
+    }
+    if (x >= x_end) return false;
+    if (x < cum) {
+      seek_round(p, x);  // first piece after the head piece
+    } else {
+      while (x >= cum + HB * cost(n)) {
+        cum += HB * cost(n);
+        ++r;
+        n = unit_tiles(p.Nq, p.Nk, p.causal, p.n_qblk - 1 - r);
+      }
+    }
+    const int w = cost(n);
+    const int k = (x - cum) / w;
+    const int base = cum + k * w + kUnitCost;  // position of iteration 0 of unit k
+    const int jb = max(0, x - base), je = min(n, x_end - base);
+    if (je <= jb) {  // the range ends inside this unit's fixed cost: no iteration left
+      x = x_end;
+      return false;
+    }
+    k_cur = k;
+    fill(p, pc, r, k, jb, je);
+    x = base + je;
+    return true;
+  }
+};
 
 // 2^x for a pair of fp32 values on the FMA pipe instead of the MUFU: a
 // Cody-Waite split x = j + f with j = round(x), f in [-1/2, 1/2], then
@@ -169,21 +388,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  volatile int* sm_job = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);  // 1: merge the unit
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- block -> (query block, head, batch); heaviest query blocks first ----
-  const int hb_count = p.Hq * p.B;
-  const int hb = blockIdx.x % hb_count;
-  const int qb = p.n_qblk - 1 - static_cast<int>(blockIdx.x / hb_count);
-  const int hq = hb % p.Hq;
-  const int b = hb / p.Hq;
-  const int hk = hq / (p.Hq / p.Hkv);
-  const int row0 = qb * kRowsPerCta;  // first row of Q0; Q1 starts kBlockM later
-  const int nt0 = kv_tiles_for(p, row0);
-  const int nt1 = kv_tiles_for(p, row0 + kBlockM);
-  const int n_kv = max(nt0, nt1);
   const int koff = p.Nk - p.Nq;  // causal diagonal offset
 
   // ---- setup ----
@@ -191,8 +399,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     for (int i = 0; i < BAR_KV_FULL; ++i) {
       uint32_t cnt = 1;
-      if ((i >= BAR_STATS && i < BAR_STATS + 2) || (i >= BAR_FSTATS && i < BAR_FSTATS + 2))
+      if ((i >= BAR_STATS && i < BAR_STATS + 2) || (i >= BAR_FSTATS && i < BAR_FSTATS + 2) ||
+          (i >= BAR_FCONS && i < BAR_FCONS + 2) || i == BAR_GRP)
         cnt = kBlockM;
+      if (i == BAR_MFREE) cnt = kMergeThreads;
       if (i >= BAR_P && i < BAR_P + 2) cnt = 2 * kBlockM;
       mbar_init(bar(i), cnt);
     }
@@ -212,216 +422,315 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const WaitGuard g{abort_flag, &g_status, p.limit_ns};
+  const WaitGuard g{smem_addr(const_cast<int*>(abort_flag)), p.limit_ns};
   const bool aligned_ok = (sbase & 1023u) == 0;  // always true by construction
 
-  // Register split, one instruction site per warpgroup.
+  // Each warpgroup executes one register-split instruction (one site per
+  // warpgroup) that directly dominates its role's code; every role then walks
+  // the same sequence of pieces with its own iterator.
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-  } else if (warp < 12) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCorrection));
-  } else {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
-  }
-
-  if (warp < 8) {
+    PieceIter pit;
+    pit.init(p);
+    Piece pc;
     // =================== softmax: one thread per query row ===================
     const int t = warp >> 2;
     const int q4 = warp & 3;
     const int rt = q4 * 32 + lane;  // row within the tile == TMEM lane
-    const int r0t = row0 + t * kBlockM;
-    const int ntt = t ? nt1 : nt0;
-    const int row = r0t + rt;
     const uint32_t tS = tmem + (static_cast<uint32_t>(q4 * 32) << 16) + C::col_s(t);
     const float c = p.c;
-    float m_raw = -INFINITY;  // running max of the raw scores
-    float m_sc = 0.f;         // m_raw * c (0 while no key was visible)
-    float l = 0.f;            // running denominator, relative to m_sc
-    for (int j = 0; j < ntt; ++j) {
-      if (!mbar_wait(bar(BAR_S + t), j & 1, g, FA2_SITE_S_READY, j)) break;
-      tc_fence_after();
-      float s[kBlockN];
-#pragma unroll
-      for (int k = 0; k < kBlockN / 32; ++k) {
-        uint32_t r[32];
-        tmem_ld32(tS + 32 * k, r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[32 * k + i] = __uint_as_float(r[i]);
-      }
-      tmem_wait_ld();
-      // causal diagonal / ragged key tail: only these tiles pay for masking
-      const int kbase = j * kBlockN;
-      const bool masked = (kbase + kBlockN > p.Nk) || (p.causal && kbase + kBlockN - 1 > r0t + koff);
-      int lim = kBlockN - 1;  // last visible column of this tile for this row
-      if (masked) {
-        lim = min(lim, p.Nk - 1 - kbase);
-        if (p.causal) lim = min(lim, row + koff - kbase);
-#pragma unroll
-        for (int i = 0; i < kBlockN; ++i)
-          if (i > lim) s[i] = -INFINITY;
-      }
-      // row max: 8 independent chains of 3-input max (max is exact in any order)
-      float mp[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mp[k] = fmaxf(s[2 * k], s[2 * k + 1]);
-#pragma unroll
-      for (int i = 16; i < kBlockN; i += 16)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mp[k] = fmax3(mp[k], s[i + 2 * k], s[i + 2 * k + 1]);
-      const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]),
-                             fmax3(mp[6], mp[7], m_raw));
-      const float m_sc_new = (mx == -INFINITY) ? 0.f : mx * c;
-      // rescale factor for what was accumulated so far: exactly 1 when the max
-      // did not move (then O is left untouched), 0 when nothing was visible yet
-      float alpha = 1.f;
-      if (mx != m_raw) alpha = (m_raw == -INFINITY) ? 0.f : ex2_approx(m_sc - m_sc_new);
-      if (j > 0) {
-        // Publish the rescale factor; the correction warps apply it to O
-        // while this thread computes the exponentials.
-        sm_alpha[t * kBlockM + rt] = alpha;
-        mbar_arrive(bar(BAR_STATS + t));
-      }
-      // p = 2^(s*c - m*c): one packed FMA per pair of scores, then ex2
-      const uint64_t cc = f2_pack(c, c), nn = f2_pack(-m_sc_new, -m_sc_new);
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // packed partial row sums (+0.0f pairs)
-      const uint32_t tP = tS;  // P (bf16) overwrites the first half of S
-      auto exp_row = [&](auto emu_tag) {
-        constexpr int kEmu = decltype(emu_tag)::value;
-#pragma unroll
-        for (int k = 0; k < kBlockN / 32; ++k) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c0 = 32 * k + 2 * i;
-            float x0, x1, e0, e1;
-            f2_unpack(f2_fma(f2_pack(s[c0], s[c0 + 1]), cc, nn), x0, x1);
-            if (i >= 16 - kEmu) {
-              exp2_poly_pair(x0, x1, e0, e1);
-            } else {
-              e0 = ex2_approx(x0);
-              e1 = ex2_approx(x1);
-            }
-            acc[i & 3] = f2_add(acc[i & 3], f2_pack(e0, e1));
-            pk[i] = pack_bf16x2(e0, e1);
-          }
-          tmem_st16(tP + 16 * k, pk);
-        }
-      };
-      if (masked)  // masked scores are -inf and must give exactly 0: MUFU only
-        exp_row(std::integral_constant<int, 0>{});
-      else
-        exp_row(std::integral_constant<int, kEmuPairs>{});
-      float sum[8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) f2_unpack(acc[i], sum[2 * i], sum[2 * i + 1]);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(BAR_P + t));
-      l = l * alpha + (((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7])));
-      m_raw = mx;
-      m_sc = m_sc_new;
-    }
-    sm_m[t * kBlockM + rt] = (m_raw == -INFINITY) ? -INFINITY : m_sc;
-    sm_l[t * kBlockM + rt] = l;
-    mbar_arrive(bar(BAR_FSTATS + t));
-  } else if (warp < 12) {
-    // ============== correction (O rescale) and epilogue warps ==============
-    const int q4 = warp & 3;
-    const int rt = q4 * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    uint32_t s_cnt = 0;      // S_t completions consumed so far (all pieces)
+    uint32_t piece_cnt = 0;  // pieces finished
     bool ok = true;
-    for (int j = 0; j < n_kv && ok; ++j) {
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (j >= (t ? nt1 : nt0)) continue;
-        if (j == 0) {  // nothing accumulated yet: O_t is ready for the first PV
-          mbar_arrive(bar(BAR_P + t));
-          continue;
-        }
-        if (!mbar_wait(bar(BAR_STATS + t), (j - 1) & 1, g, FA2_SITE_STATS_READY, j)) {
+    while (ok && pit.next(p, pc)) {
+      const int ntt = t ? pc.a1 : pc.a0;
+      const int r0t = pc.qb * kRowsPerCta + t * kBlockM;
+      const int row = r0t + rt;
+      float m_raw = -INFINITY;  // running max of the raw scores
+      float m_sc = 0.f;         // m_raw * c (0 while no key was visible)
+      float l = 0.f;            // running denominator, relative to m_sc
+      for (int jj = 0; jj < ntt; ++jj) {
+        const int j = pc.jb + jj;  // K/V tile of the unit
+        if (!mbar_wait_warp(bar(BAR_S + t), s_cnt & 1, g, FA2_SITE_S_READY, j)) {
           ok = false;
           break;
         }
-        const float alpha = sm_alpha[t * kBlockM + rt];
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          // the previous PV into O_t completed before S_t(j) did, which the
-          // softmax threads waited for before publishing alpha
-          tc_fence_after();
-          const uint32_t tO = tmem + lane_off + C::col_o(t);
-          const uint64_t aa = f2_pack(alpha, alpha);
-#pragma unroll 1
-          for (int ch = 0; ch < D / 16; ++ch) {
-            uint32_t r[16];
-            tmem_ld16(tO + 16 * ch, r);
-            tmem_wait_ld();
+        ++s_cnt;
+        tc_fence_after();
+        float s[kBlockN];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float lo, hi;
-              f2_unpack(f2_mul(f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), aa), lo, hi);
-              r[2 * i] = __float_as_uint(lo);
-              r[2 * i + 1] = __float_as_uint(hi);
-            }
-            tmem_st16(tO + 16 * ch, r);
-          }
-          tmem_wait_st();
+        for (int k = 0; k < kBlockN / 32; ++k) {
+          uint32_t r[32];
+          tmem_ld32(tS + 32 * k, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[32 * k + i] = __uint_as_float(r[i]);
         }
+        tmem_wait_ld();
+        // causal diagonal / ragged key tail: only these tiles pay for masking
+        const int kbase = j * kBlockN;
+        const bool masked = (kbase + kBlockN > p.Nk) || (p.causal && kbase + kBlockN - 1 > r0t + koff);
+        int lim = kBlockN - 1;  // last visible column of this tile for this row
+        if (masked) {
+          lim = min(lim, p.Nk - 1 - kbase);
+          if (p.causal) lim = min(lim, row + koff - kbase);
+#pragma unroll
+          for (int i = 0; i < kBlockN; ++i)
+            if (i > lim) s[i] = -INFINITY;
+        }
+        // row max: 8 independent chains of 3-input max (max is exact in any order)
+        float mp[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mp[k] = fmaxf(s[2 * k], s[2 * k + 1]);
+#pragma unroll
+        for (int i = 16; i < kBlockN; i += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mp[k] = fmax3(mp[k], s[i + 2 * k], s[i + 2 * k + 1]);
+        const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]),
+                               fmax3(mp[6], mp[7], m_raw));
+        const float m_sc_new = (mx == -INFINITY) ? 0.f : mx * c;
+        // rescale factor for what was accumulated so far: exactly 1 when the max
+        // did not move (then O is left untouched), 0 when nothing was visible yet
+        float alpha = 1.f;
+        if (mx != m_raw) alpha = (m_raw == -INFINITY) ? 0.f : ex2_approx(m_sc - m_sc_new);
+        if (jj > 0) {
+          // Publish the rescale factor; the correction warps apply it to O
+          // while this thread computes the exponentials.
+          sm_alpha[t * kBlockM + rt] = alpha;
+          mbar_arrive(bar(BAR_STATS + t));
+        }
+        // p = 2^(s*c - m*c): one packed FMA per pair of scores, then ex2
+        const uint64_t cc = f2_pack(c, c), nn = f2_pack(-m_sc_new, -m_sc_new);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // packed partial row sums (+0.0f pairs)
+        const uint32_t tP = tS;  // P (bf16) overwrites the first half of S
+        auto exp_row = [&](auto emu_tag) {
+          constexpr int kEmu = decltype(emu_tag)::value;
+#pragma unroll
+          for (int k = 0; k < kBlockN / 32; ++k) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int c0 = 32 * k + 2 * i;
+              float x0, x1, e0, e1;
+              f2_unpack(f2_fma(f2_pack(s[c0], s[c0 + 1]), cc, nn), x0, x1);
+              if (i >= 16 - kEmu) {
+                exp2_poly_pair(x0, x1, e0, e1);
+              } else {
+                e0 = ex2_approx(x0);
+                e1 = ex2_approx(x1);
+              }
+              acc[i & 3] = f2_add(acc[i & 3], f2_pack(e0, e1));
+              pk[i] = pack_bf16x2(e0, e1);
+            }
+            tmem_st16(tP + 16 * k, pk);
+          }
+        };
+        if (masked)  // masked scores are -inf and must give exactly 0: MUFU only
+          exp_row(std::integral_constant<int, 0>{});
+        else
+          exp_row(std::integral_constant<int, kEmuPairs>{});
+        float sum[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) f2_unpack(acc[i], sum[2 * i], sum[2 * i + 1]);
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(BAR_P + t));
+        l = l * alpha + (((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7])));
+        m_raw = mx;
+        m_sc = m_sc_new;
       }
+      if (!ok) break;
+      // final statistics of this piece; the previous piece's must have been read
+      if (piece_cnt > 0 &&
+          !mbar_wait_warp(bar(BAR_FCONS + t), (piece_cnt - 1) & 1, g, FA2_SITE_FINAL_STATS, piece_cnt)) {
+        ok = false;
+        break;
+      }
+      sm_m[t * kBlockM + rt] = (m_raw == -INFINITY) ? -INFINITY : m_sc;
+      sm_l[t * kBlockM + rt] = l;
+      mbar_arrive(bar(BAR_FSTATS + t));
+      ++piece_cnt;
     }
-    // epilogue: O / l -> bf16, LSE = ln(sum exp(scale * s))
+  } else if (warp < 12) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCorrection));
+    PieceIter pit;
+    pit.init(p);
+    Piece pc;
+    // ============== correction (O rescale) and epilogue warps ==============
+    const int q4 = warp & 3;
+    const int rt = q4 * 32 + lane;
+    const int ct = threadIdx.x - 256;  // 0..127 within the correction warps
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    // parities of the phases consumed so far: bit t = STATS_t, bit 2 + t =
+    // OFINAL_t, bit 4 = FSTATS (one per piece), bit 5 = GRP and bit 6 =
+    // MFREE (one per split piece); bit 7: a merge job was posted before
+    uint32_t ph = 0;
+    bool ok = true;
+
+    while (ok && pit.next(p, pc)) {
+      const int n_p = pc.je - pc.jb;
+      for (int jj = 0; jj < n_p && ok; ++jj) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (jj >= (t ? pc.a1 : pc.a0)) continue;
+          if (jj == 0) {  // nothing accumulated yet: O_t (read by the last epilogue) is free
+            tc_fence_before();
+            mbar_arrive(bar(BAR_P + t));
+            continue;
+          }
+          if (!mbar_wait_warp(bar(BAR_STATS + t), (ph >> t) & 1, g, FA2_SITE_STATS_READY, pc.jb + jj)) {
+            ok = false;
+            break;
+          }
+          ph ^= 1u << t;
+          const float alpha = sm_alpha[t * kBlockM + rt];
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+            // the previous PV into O_t completed before S_t(j) did, which the
+            // softmax threads waited for before publishing alpha
+            tc_fence_after();
+            const uint32_t tO = tmem + lane_off + C::col_o(t);
+            const uint64_t aa = f2_pack(alpha, alpha);
 #pragma unroll 1
-    for (int t = 0; t < 2; ++t) {
-      const int row = row0 + t * kBlockM + rt;
-      const bool valid = row < p.Nq;
-      float inv_l = 0.f, lse = -INFINITY;
-      bool have_o = false;
-      if ((t ? nt1 : nt0) > 0 && ok) {
-        if (!mbar_wait(bar(BAR_OFINAL + t), 0, g, FA2_SITE_O_FINAL, t) ||
-            !mbar_wait(bar(BAR_FSTATS + t), 0, g, FA2_SITE_FINAL_STATS, t)) {
+            for (int ch = 0; ch < D / 16; ++ch) {
+              uint32_t r[16];
+              tmem_ld16(tO + 16 * ch, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                float lo, hi;
+                f2_unpack(f2_mul(f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), aa), lo, hi);
+                r[2 * i] = __float_as_uint(lo);
+                r[2 * i + 1] = __float_as_uint(hi);
+              }
+              tmem_st16(tO + 16 * ch, r);
+            }
+            tmem_wait_st();
+          }
+          tc_fence_before();
+          mbar_arrive(bar(BAR_P + t));
+        }
+      }
+      if (!ok) break;
+      pit.coords(p, pc);
+      pit.split_info(p, pc);
+
+      // ---- epilogue of the piece, tile by tile: a whole unit is normalised
+      // and stored; a piece of a split unit publishes its partial instead ----
+      float* part = nullptr;
+      if (pc.split)
+        part = p.ws + static_cast<size_t>(2 * (pc.slot + pc.index) + (pc.index == 0 ? 1 : 0)) *
+                          C::kPieceFloats;
+#pragma unroll 1
+      for (int t = 0; t < 2; ++t) {
+        const bool have = (t ? pc.a1 : pc.a0) > 0;  // warp-uniform: tcgen05.ld needs the whole warp
+        if (have) {
+          if (!mbar_wait_warp(bar(BAR_OFINAL + t), (ph >> (2 + t)) & 1, g, FA2_SITE_O_FINAL, t)) {
+            ok = false;
+            break;
+          }
+          ph ^= 4u << t;
+        }
+        if (!mbar_wait_warp(bar(BAR_FSTATS + t), (ph >> 4) & 1, g, FA2_SITE_FINAL_STATS, t)) {
           ok = false;
-        } else {
-          tc_fence_after();
-          const float m_sc = sm_m[t * kBlockM + rt];
-          const float l = sm_l[t * kBlockM + rt];
+          break;
+        }
+        const float m_sc = sm_m[t * kBlockM + rt];
+        const float l = sm_l[t * kBlockM + rt];
+        mbar_arrive(bar(BAR_FCONS + t));
+        tc_fence_after();
+        const uint32_t tO = tmem + lane_off + C::col_o(t);
+        if (!pc.split) {
+          // single division per row, bf16 O, LSE = ln(sum exp(scale * s))
+          const int row = pc.qb * kRowsPerCta + t * kBlockM + rt;
+          const bool valid = row < p.Nq;
+          float inv_l = 0.f, lse = -INFINITY;
           if (l > 0.f) {
             inv_l = 1.f / l;
             lse = (m_sc + log2f(l)) * 0.69314718055994530942f;
           }
-          have_o = true;
-        }
-      }
-      __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Nq + row) * p.Hq + hq) * D;
-      const uint32_t tO = tmem + lane_off + C::col_o(t);
+          __nv_bfloat16* orow = p.o + ((static_cast<size_t>(pc.b) * p.Nq + row) * p.Hq + pc.hq) * D;
 #pragma unroll 1
-      for (int ch = 0; ch < D / 16; ++ch) {
-        uint32_t r[16];
-        if (have_o) {
-          tmem_ld16(tO + 16 * ch, r);
-          tmem_wait_ld();
+          for (int ch = 0; ch < D / 16; ++ch) {
+            uint32_t r[16];
+            if (have) {
+              tmem_ld16(tO + 16 * ch, r);
+              tmem_wait_ld();
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) r[i] = 0u;
+            }
+            uint4 w0, w1;
+            w0.x = pack_bf16x2(__uint_as_float(r[0]) * inv_l, __uint_as_float(r[1]) * inv_l);
+            w0.y = pack_bf16x2(__uint_as_float(r[2]) * inv_l, __uint_as_float(r[3]) * inv_l);
+            w0.z = pack_bf16x2(__uint_as_float(r[4]) * inv_l, __uint_as_float(r[5]) * inv_l);
+            w0.w = pack_bf16x2(__uint_as_float(r[6]) * inv_l, __uint_as_float(r[7]) * inv_l);
+            w1.x = pack_bf16x2(__uint_as_float(r[8]) * inv_l, __uint_as_float(r[9]) * inv_l);
+            w1.y = pack_bf16x2(__uint_as_float(r[10]) * inv_l, __uint_as_float(r[11]) * inv_l);
+            w1.z = pack_bf16x2(__uint_as_float(r[12]) * inv_l, __uint_as_float(r[13]) * inv_l);
+            w1.w = pack_bf16x2(__uint_as_float(r[14]) * inv_l, __uint_as_float(r[15]) * inv_l);
+            if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + 16 * ch);
+              dst[0] = w0;
+              dst[1] = w1;
+            }
+          }
+          if (valid) p.lse[(static_cast<size_t>(pc.b) * p.Hq + pc.hq) * p.Nq + row] = lse;
         } else {
+          // partial: O unnormalised (fp32), in 16-column chunks of 128 rows so
+          // a warp's store covers 32 consecutive rows (2 KiB contiguous)
+          if (have) {
+#pragma unroll 1
+            for (int ch = 0; ch < D / 16; ++ch) {
+              uint32_t r[16];
+              tmem_ld16(tO + 16 * ch, r);
+              tmem_wait_ld();
+              float4* dst = reinterpret_cast<float4*>(part + C::part_o(t, ch, rt));
 #pragma unroll
-          for (int i = 0; i < 16; ++i) r[i] = 0u;
-        }
-        uint4 w[2];
-        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          wp[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 16 * ch);
-          dst[0] = w[0];
-          dst[1] = w[1];
+              for (int i = 0; i < 4; ++i)
+                __stcg(dst + i, make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                            __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
+            }
+          }
+          __stcg(part + C::part_m(t, rt), m_sc);
+          __stcg(part + C::part_l(t, rt), have ? l : 0.f);
         }
       }
-      if (valid) p.lse[(static_cast<size_t>(b) * p.Hq + hq) * p.Nq + row] = lse;
+      if (!ok) break;
+      ph ^= 16u;
+      if (!pc.split) continue;
+
+      // ---- split piece: take a ticket once all 128 rows are published and
+      // hand the outcome to the merge warps (the last piece's CTA merges) ----
+      __threadfence();
+      mbar_arrive(bar(BAR_GRP));
+      if (ct == 0) {
+        if (!mbar_wait(bar(BAR_GRP), (ph >> 5) & 1, g, FA2_SITE_MERGE, 0)) {
+          ok = false;
+        } else {
+          const int ticket = atomicAdd(p.ws_ctr + pc.slot, 1);
+          if ((ph & 128u) && !mbar_wait(bar(BAR_MFREE), (ph >> 6) & 1, g, FA2_SITE_MERGE, 1)) {
+            ok = false;
+          } else {
+            *sm_job = (ticket == pc.npieces - 1) ? 1 : 0;
+            mbar_arrive(bar(BAR_MJOB));
+          }
+        }
+      }
+      if (ph & 128u) ph ^= 64u;  // the MFREE phase the last job completed
+      ph ^= 32u;
+      ph |= 128u;
+      if (warp == 8) ok = __all_sync(0xffffffffu, ok);  // keep the warp converged
     }
-  } else if (warp == 12) {
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+    PieceIter pit;
+    pit.init(p);
+    Piece pc;
+   if (warp == 12) {
     // ============================ MMA issuer warp ============================
     // The whole warp follows the schedule (warp-uniform waits and descriptor
     // arithmetic); one elected lane -- always the same one in a converged warp,
     // so its commits cover its own MMAs -- issues each group of tcgen05
-    // instructions (8 MMAs and their commit) inside a single elected block.
+    // instructions (MMAs and their commits) inside a single elected block.
     // Measured on B200: a group issued this way takes ~23 cycles per MMA and
     // runs ahead of the tensor core, while a per-MMA elect/warp-sync costs
     // 50-60 cycles each and a single divergent lane is slower still when the
@@ -431,8 +740,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idPV = idesc_bf16_f32(kBlockM, D, true, false);
       const uint32_t sQ = sbase + C::kOffQ;
       const uint32_t sKV = sbase + C::kOffKV;
-      auto stage_of = [&](int it) { return it % C::kStages; };
-      auto phase_of = [&](int it) { return static_cast<uint32_t>((it / C::kStages) & 1); };
+      auto stage_of = [&](uint32_t it) { return static_cast<int>(it % C::kStages); };
+      auto phase_of = [&](uint32_t it) { return (it / C::kStages) & 1u; };
+      auto free_of = [&](uint32_t it) { return bar(BAR_KV_FULL + C::kStages + stage_of(it)); };
       // The start-address field is the low 14 bits of the descriptor (address
       // >> 4, below 2^14 for any shared-memory address), so advancing along K
       // inside a tile is a plain add of (byte offset >> 4).
@@ -443,94 +753,104 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (elect_one()) umma_commit(b);
         __syncwarp();
       };
-      // One elected block per tile and KV step: O_t += P_t V_j, then (if any)
-      // S_t(j+1) = Q_t K_{j+1}^T, then the commits that publish completion.
-      // S_t(j+1) overwrites the TMEM columns that held P_t(j); it is issued by
-      // the same thread after the PV that reads them, and one thread's tcgen05
-      // MMAs execute in issue order.
-      auto issue_block = [&](int t, int j, bool pv, bool s_next, uint32_t c_pv1, uint32_t c_pv2,
-                             uint32_t c_s1, uint32_t c_s2) {
-        const uint32_t dS = tmem + C::col_s(t), dO = tmem + C::col_o(t);
-        const uint64_t bV = dV + ((stage_of(2 * j + 1) * C::kTileBytes) >> 4);
+      // S_t = Q_t K^T with the K tile of ring item itK, then commits
+      auto issue_s = [&](int t, uint32_t itK, uint32_t c1, uint32_t c2, uint32_t c3) {
+        const uint32_t dS = tmem + C::col_s(t);
         const uint64_t a0 = dQ + ((t * C::kTileBytes) >> 4);
-        const uint64_t bK = dK + ((stage_of(2 * j + 2) * C::kTileBytes) >> 4);
+        const uint64_t bK = dK + ((stage_of(itK) * C::kTileBytes) >> 4);
         if (elect_one()) {
-          if (pv) {
+          // K advances 32 bytes inside a 128-byte swizzle atom, then jumps to
+          // the next 64-column chunk.  (The empty asm makes the per-MMA
+          // descriptors opaque, so the compiler derives them here instead of
+          // keeping all of them live across the whole schedule.)
+          uint64_t da = a0, db = bK;
+          asm volatile("" : "+l"(da), "+l"(db));
 #pragma unroll
-            for (int kk = 0; kk < kBlockN / 16; ++kk)
-              umma_ts(dO, dS + kk * 8, bV + ((kk * 16 * kSwizzleBytes) >> 4), idPV,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-            if (c_pv1) umma_commit(c_pv1);
-            if (c_pv2) umma_commit(c_pv2);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            umma_ss(dS, da, db, idS, kk > 0 ? 1u : 0u);
+            const uint32_t step = ((kk & 3) == 3) ? (kChunkBytes - 3 * 32) >> 4 : 32 >> 4;
+            da += step;
+            db += step;
           }
-          if (s_next) {
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
-              umma_ss(dS, a0 + off, bK + off, idS, kk > 0 ? 1u : 0u);
-            }
-            if (c_s1) umma_commit(c_s1);
-            if (c_s2) umma_commit(c_s2);
-          }
+          if (c1) umma_commit(c1);
+          if (c2) umma_commit(c2);
+          if (c3) umma_commit(c3);
         }
         __syncwarp();
       };
-      // S_t(0)
-      auto issue_s0 = [&](int t, uint32_t c2) {
-        const uint32_t dS = tmem + C::col_s(t);
-        const uint64_t a0 = dQ + ((t * C::kTileBytes) >> 4);
-        const uint64_t bK = dK + ((stage_of(0) * C::kTileBytes) >> 4);
+      // O_t (+)= P_t V with the V tile of ring item itV, then commits
+      auto issue_pv = [&](int t, uint32_t itV, bool acc, uint32_t c1, uint32_t c2) {
+        const uint32_t dS = tmem + C::col_s(t), dO = tmem + C::col_o(t);
+        const uint64_t bV = dV + ((stage_of(itV) * C::kTileBytes) >> 4);
         if (elect_one()) {
+          uint64_t db = bV;
+          asm volatile("" : "+l"(db));
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
-            umma_ss(dS, a0 + off, bK + off, idS, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kBlockN / 16; ++kk) {
+            umma_ts(dO, dS + kk * 8, db, idPV, (acc || kk > 0) ? 1u : 0u);
+            db += (16 * kSwizzleBytes) >> 4;  // next 16 keys
           }
-          umma_commit(bar(BAR_S + t));
+          if (c1) umma_commit(c1);
           if (c2) umma_commit(c2);
         }
         __syncwarp();
       };
-      auto free_of = [&](int it) { return bar(BAR_KV_FULL + C::kStages + stage_of(it)); };
+      uint32_t itb = 0;           // ring item of the current piece's first K tile
+      uint32_t q_cnt = 0;         // pieces whose Q was waited for
+      uint32_t p_cnt[2] = {0, 0}; // P_t phases consumed
       bool ok = true;
-      if (nt0 > 0) ok = mbar_wait_warp(bar(BAR_Q + 0), 0, g, FA2_SITE_Q_LOADED, 0);
-      if (ok && nt1 > 0) ok = mbar_wait_warp(bar(BAR_Q + 1), 0, g, FA2_SITE_Q_LOADED, 1);
-      if (ok && n_kv > 0) {
-        ok = mbar_wait_warp(bar(BAR_KV_FULL + stage_of(0)), phase_of(0), g, FA2_SITE_KV_LOADED, 0);
-        if (ok) {
-          tc_fence_after();
-          if (nt0 > 0) issue_s0(0, nt1 > 0 ? 0u : free_of(0));
-          if (nt1 > 0) issue_s0(1, free_of(0));
-        }
-      }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int itV = 2 * j + 1, itK = 2 * j + 2;
-        const bool next = (j + 1 < n_kv);
-        // operands of this step (normally landed long ago); checked while the
-        // tensor pipe still holds the previous block
-        if (!mbar_wait_warp(bar(BAR_KV_FULL + stage_of(itV)), phase_of(itV), g, FA2_SITE_KV_LOADED, j)) break;
-        if (next && !mbar_wait_warp(bar(BAR_KV_FULL + stage_of(itK)), phase_of(itK), g,
-                                    FA2_SITE_KV_LOADED, j + 1))
+      while (ok && pit.next(p, pc)) {
+        const int n_p = pc.je - pc.jb;
+        const int a0 = pc.a0, a1 = pc.a1;
+        if (!mbar_wait_warp(bar(BAR_Q), q_cnt & 1, g, FA2_SITE_Q_LOADED, q_cnt)) break;
+        ++q_cnt;
+        auto itK = [&](int jj) { return itb + 2u * static_cast<uint32_t>(jj); };
+        auto itV = [&](int jj) { return itb + 2u * static_cast<uint32_t>(jj) + 1u; };
+        // S_t of the piece's first K/V tile; K is free after the last S on it
+        if (!mbar_wait_warp(bar(BAR_KV_FULL + stage_of(itK(0))), phase_of(itK(0)), g,
+                            FA2_SITE_KV_LOADED, pc.jb))
           break;
-        // tile 0: PV0(j) and S0(j+1); V_j / K_{j+1} are freed here when tile 1 has no use for them
-        if (j < nt0) {
-          if (!mbar_wait_warp(bar(BAR_P + 0), j & 1, g, FA2_SITE_P_READY, j)) break;
-          tc_fence_after();
-          issue_block(0, j, true, j + 1 < nt0, j == nt0 - 1 ? bar(BAR_OFINAL + 0) : 0u,
-                      j >= nt1 ? free_of(itV) : 0u, bar(BAR_S + 0), j + 1 >= nt1 ? free_of(itK) : 0u);
+        tc_fence_after();
+        const uint32_t qfree0 = (n_p == 1) ? bar(BAR_QFREE) : 0u;
+        if (a0 > 0) issue_s(0, itK(0), bar(BAR_S + 0), a1 > 0 ? 0u : free_of(itK(0)), a1 > 0 ? 0u : qfree0);
+        if (a1 > 0) issue_s(1, itK(0), bar(BAR_S + 1), free_of(itK(0)), qfree0);
+        for (int jj = 0; jj < n_p && ok; ++jj) {
+          const bool next = (jj + 1 < n_p);
+          // operands of this step (normally landed long ago); checked while the
+          // tensor pipe still holds the previous block
+          if (!mbar_wait_warp(bar(BAR_KV_FULL + stage_of(itV(jj))), phase_of(itV(jj)), g,
+                              FA2_SITE_KV_LOADED, pc.jb + jj))
+            break;
+          if (next && !mbar_wait_warp(bar(BAR_KV_FULL + stage_of(itK(jj + 1))), phase_of(itK(jj + 1)), g,
+                                      FA2_SITE_KV_LOADED, pc.jb + jj + 1))
+            break;
+          // the last S of the piece frees the Q buffer for the next piece
+          const uint32_t qfree = (jj + 2 == n_p) ? bar(BAR_QFREE) : 0u;
+          // tile 0: PV0(j) and S0(j+1); V_j / K_{j+1} are freed here when tile 1 has no use for them
+          if (jj < a0) {
+            if (!mbar_wait_warp(bar(BAR_P + 0), p_cnt[0] & 1, g, FA2_SITE_P_READY, pc.jb + jj)) break;
+            ++p_cnt[0];
+            tc_fence_after();
+            issue_pv(0, itV(jj), jj > 0, jj == a0 - 1 ? bar(BAR_OFINAL + 0) : 0u,
+                     jj >= a1 ? free_of(itV(jj)) : 0u);
+            if (jj + 1 < a0)
+              issue_s(0, itK(jj + 1), bar(BAR_S + 0), jj + 1 >= a1 ? free_of(itK(jj + 1)) : 0u,
+                      jj + 1 >= a1 ? qfree : 0u);
+          }
+          // tile 1: PV1(j) and S1(j+1); the last use of V_j and K_{j+1}
+          if (jj < a1) {
+            if (!mbar_wait_warp(bar(BAR_P + 1), p_cnt[1] & 1, g, FA2_SITE_P_READY, pc.jb + jj)) break;
+            ++p_cnt[1];
+            tc_fence_after();
+            issue_pv(1, itV(jj), jj > 0, free_of(itV(jj)), jj == a1 - 1 ? bar(BAR_OFINAL + 1) : 0u);
+            if (jj + 1 < a1) issue_s(1, itK(jj + 1), bar(BAR_S + 1), free_of(itK(jj + 1)), qfree);
+          }
         }
-        // tile 1: PV1(j) and S1(j+1); the last use of V_j and K_{j+1}
-        if (j < nt1) {
-          if (!mbar_wait_warp(bar(BAR_P + 1), j & 1, g, FA2_SITE_P_READY, j)) break;
-          tc_fence_after();
-          issue_block(1, j, true, j + 1 < nt1, free_of(itV), j == nt1 - 1 ? bar(BAR_OFINAL + 1) : 0u,
-                      bar(BAR_S + 1), free_of(itK));
-        }
+        itb += 2u * static_cast<uint32_t>(n_p);
       }
       // drain: every MMA issued above has completed before TMEM is released
       // (not cut short by the abort flag: tensor-core work always finishes)
-      volatile int no_abort = 0;
-      const WaitGuard drain{&no_abort, &g_status, p.limit_ns};
+      const WaitGuard drain{0u, p.limit_ns};
       commit(bar(BAR_DONE));
       mbar_wait_warp(bar(BAR_DONE), 0, drain, FA2_SITE_MMA_DRAIN, 0);
     }
@@ -539,50 +859,161 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (aligned_ok) {
       const uint32_t sQ = sbase + C::kOffQ;
       const uint32_t sKV = sbase + C::kOffKV;
-#pragma unroll 1
-      for (int t = 0; t < 2; ++t) {
-        if ((t ? nt1 : nt0) == 0) continue;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(bar(BAR_Q + t), C::kTileBytes);
-#pragma unroll
-          for (int ch = 0; ch < C::kChunks; ++ch)
-            tma_load_4d(sQ + t * C::kTileBytes + ch * kChunkBytes, &tmQ, bar(BAR_Q + t), ch * 64, hq,
-                        row0 + t * kBlockM, b);
-        }
-        __syncwarp();
-      }
-      int issued = 0;
+      uint32_t it = 0;       // ring items issued
+      uint32_t pieces = 0;   // pieces whose Q was loaded
       bool ok = true;
-      for (int it = 0; it < 2 * n_kv; ++it) {
-        const int st = it % C::kStages;
-        if (it >= C::kStages &&
-            !mbar_wait_warp(bar(BAR_KV_FULL + C::kStages + st), ((it / C::kStages) & 1) ^ 1, g,
-                            FA2_SITE_KV_FREE, it)) {
+      while (ok && pit.next(p, pc)) {
+        const int hk = pc.hq / (p.Hq / p.Hkv);
+        // Q of this piece, once the previous piece's last S MMA released the buffer
+        if (pieces > 0 && !mbar_wait_warp(bar(BAR_QFREE), (pieces - 1) & 1, g, FA2_SITE_Q_LOADED, pieces)) {
           ok = false;
           break;
         }
         if (elect_one()) {
-          mbar_arrive_expect_tx(bar(BAR_KV_FULL + st), C::kTileBytes);
-          const CUtensorMap* map = (it & 1) ? &tmV : &tmK;
+          const uint32_t bytes = (pc.a0 > 0 ? C::kTileBytes : 0) + (pc.a1 > 0 ? C::kTileBytes : 0);
+          mbar_arrive_expect_tx(bar(BAR_Q), bytes);
+#pragma unroll 1
+          for (int t = 0; t < 2; ++t) {
+            if ((t ? pc.a1 : pc.a0) == 0) continue;
 #pragma unroll
-          for (int ch = 0; ch < C::kChunks; ++ch)
-            tma_load_4d(sKV + st * C::kTileBytes + ch * kChunkBytes, map, bar(BAR_KV_FULL + st),
-                        ch * 64, hk, (it >> 1) * kBlockN, b);
+            for (int ch = 0; ch < C::kChunks; ++ch)
+              tma_load_4d(sQ + t * C::kTileBytes + ch * kChunkBytes, &tmQ, bar(BAR_Q), ch * 64, pc.hq,
+                          pc.qb * kRowsPerCta + t * kBlockM, pc.b);
+          }
         }
         __syncwarp();
-        issued = it + 1;
+        ++pieces;
+        for (int j = pc.jb; j < pc.je && ok; ++j) {
+#pragma unroll 1
+          for (int kv = 0; kv < 2; ++kv, ++it) {
+            const int st = static_cast<int>(it % C::kStages);
+            if (it >= static_cast<uint32_t>(C::kStages) &&
+                !mbar_wait_warp(bar(BAR_KV_FULL + C::kStages + st), ((it / C::kStages) & 1) ^ 1, g,
+                                FA2_SITE_KV_FREE, static_cast<int>(it))) {
+              ok = false;
+              break;
+            }
+            if (elect_one()) {
+              mbar_arrive_expect_tx(bar(BAR_KV_FULL + st), C::kTileBytes);
+              const CUtensorMap* map = kv ? &tmV : &tmK;
+#pragma unroll
+              for (int ch = 0; ch < C::kChunks; ++ch)
+                tma_load_4d(sKV + st * C::kTileBytes + ch * kChunkBytes, map, bar(BAR_KV_FULL + st),
+                            ch * 64, hk, j * kBlockN, pc.b);
+            }
+            __syncwarp();
+          }
+        }
       }
       if (!ok) {
         // Give the copies already in flight time to land before the CTA exits.
-        volatile int no_abort = 0;
-        const WaitGuard drain{&no_abort, &g_status, p.limit_ns};
-        for (int it = (issued > C::kStages ? issued - C::kStages : 0); it < issued; ++it)
-          mbar_wait_warp(bar(BAR_KV_FULL + it % C::kStages), (it / C::kStages) & 1, drain,
-                         FA2_SITE_LOAD_DRAIN, it);
-        if (nt0 > 0) mbar_wait_warp(bar(BAR_Q + 0), 0, drain, FA2_SITE_LOAD_DRAIN, 0);
-        if (nt1 > 0) mbar_wait_warp(bar(BAR_Q + 1), 0, drain, FA2_SITE_LOAD_DRAIN, 1);
+        const WaitGuard drain{0u, p.limit_ns};
+        for (uint32_t i = (it > static_cast<uint32_t>(C::kStages) ? it - C::kStages : 0u); i < it; ++i)
+          mbar_wait_warp(bar(BAR_KV_FULL + i % C::kStages), (i / C::kStages) & 1, drain,
+                         FA2_SITE_LOAD_DRAIN, static_cast<int>(i));
+        if (pieces > 0) mbar_wait_warp(bar(BAR_Q), (pieces - 1) & 1, drain, FA2_SITE_LOAD_DRAIN, 0);
       }
     }
+   } else {
+    // ===================== merge warps (14-15, 64 threads) =====================
+    const int mt = threadIdx.x - (kThreads - kMergeThreads);  // 0..63
+    // Units with no K/V tile at all (causal, Nq > Nk): O = 0, LSE = -inf.
+    // They form a suffix of the unit order; CTAs share them round robin.
+    {
+      const int HB = p.B * p.Hq;
+      int r0 = 0;  // first round of empty units
+      while (r0 < p.n_qblk && unit_tiles(p.Nq, p.Nk, p.causal, p.n_qblk - 1 - r0) > 0) ++r0;
+      const int nz = (p.n_qblk - r0) * HB;
+      const int z0 = p.streamk ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x) - r0 * HB;
+      const int dz = p.streamk ? p.G : nz;  // unit mode: CTA u owns unit u only
+      for (int z = z0; z >= 0 && z < nz; z += dz) {
+        const int rr = r0 + z / HB, k = z % HB, qb = p.n_qblk - 1 - rr;
+        const int b = k / p.Hq, hq = k % p.Hq;
+        for (int i = mt; i < kRowsPerCta * (D / 8); i += kMergeThreads) {
+          const int row = qb * kRowsPerCta + i / (D / 8);
+          if (row >= p.Nq) continue;
+          reinterpret_cast<uint4*>(p.o + ((static_cast<size_t>(b) * p.Nq + row) * p.Hq + hq) * D)[i % (D / 8)] =
+              make_uint4(0u, 0u, 0u, 0u);
+          if (i % (D / 8) == 0) p.lse[(static_cast<size_t>(b) * p.Hq + hq) * p.Nq + row] = -INFINITY;
+        }
+      }
+    }
+    // Split units: for each split piece of this CTA the correction warps post
+    // whether it was the unit's last piece to publish; if so, merge all its
+    // partials (mergeable statistics: m = max m_i, l = sum l_i 2^(m_i - m),
+    // O = sum O_i 2^(m_i - m) / l), summing in piece order so the result does
+    // not depend on which CTA finished last.
+    uint32_t jobs = 0;
+    bool ok = true;
+    while (ok && pit.next(p, pc)) {
+      pit.split_info(p, pc);
+      if (!pc.split) continue;
+      if (!mbar_wait_warp(bar(BAR_MJOB), jobs & 1, g, FA2_SITE_MERGE, 2)) {
+        ok = false;
+        break;
+      }
+      const bool last = *sm_job != 0;
+      mbar_arrive(bar(BAR_MFREE));
+      ++jobs;
+      if (!last) continue;
+      __threadfence();
+      pit.coords(p, pc);
+      const float* ws = p.ws;
+      asm volatile("" : "+l"(ws));  // keep the address arithmetic here, out of the piece loop
+      auto part = [&](int q) {
+        return ws + static_cast<size_t>(2 * (pc.slot + q) + (q == 0 ? 1 : 0)) * C::kPieceFloats;
+      };
+#pragma unroll 1
+      for (int rr = mt; rr < kRowsPerCta; rr += kMergeThreads) {
+        const int t = rr / kBlockM, rt = rr % kBlockM;
+        const int row = pc.qb * kRowsPerCta + rr;
+        float m_tot = -INFINITY;
+#pragma unroll 1
+        for (int q = 0; q < pc.npieces; ++q)
+          if (__ldcg(part(q) + C::part_l(t, rt)) > 0.f) m_tot = fmaxf(m_tot, __ldcg(part(q) + C::part_m(t, rt)));
+        float l_tot = 0.f;
+#pragma unroll 1
+        for (int q = 0; q < pc.npieces; ++q) {
+          const float lq = __ldcg(part(q) + C::part_l(t, rt));
+          if (lq > 0.f) l_tot = fmaf(lq, ex2_approx(__ldcg(part(q) + C::part_m(t, rt)) - m_tot), l_tot);
+        }
+        if (row >= p.Nq) continue;
+        const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
+        __nv_bfloat16* orow = p.o + ((static_cast<size_t>(pc.b) * p.Nq + row) * p.Hq + pc.hq) * D;
+#pragma unroll 1
+        for (int h = 0; h < D / 8; ++h) {  // 8 columns (half a stored chunk) at a time
+          float acc[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 1
+          for (int q = 0; q < pc.npieces; ++q) {
+            const float lq = __ldcg(part(q) + C::part_l(t, rt));
+            if (!(lq > 0.f)) continue;
+            const float wq = ex2_approx(__ldcg(part(q) + C::part_m(t, rt)) - m_tot);
+            const float4* src = reinterpret_cast<const float4*>(part(q) + C::part_o(t, h >> 1, rt) + 8 * (h & 1));
+            const float4 f0 = __ldcg(src), f1 = __ldcg(src + 1);
+            acc[0] = fmaf(wq, f0.x, acc[0]);
+            acc[1] = fmaf(wq, f0.y, acc[1]);
+            acc[2] = fmaf(wq, f0.z, acc[2]);
+            acc[3] = fmaf(wq, f0.w, acc[3]);
+            acc[4] = fmaf(wq, f1.x, acc[4]);
+            acc[5] = fmaf(wq, f1.y, acc[5]);
+            acc[6] = fmaf(wq, f1.z, acc[6]);
+            acc[7] = fmaf(wq, f1.w, acc[7]);
+          }
+          uint4 w;
+          w.x = pack_bf16x2(acc[0] * inv_l, acc[1] * inv_l);
+          w.y = pack_bf16x2(acc[2] * inv_l, acc[3] * inv_l);
+          w.z = pack_bf16x2(acc[4] * inv_l, acc[5] * inv_l);
+          w.w = pack_bf16x2(acc[6] * inv_l, acc[7] * inv_l);
+          reinterpret_cast<uint4*>(orow)[h] = w;
+        }
+        p.lse[(static_cast<size_t>(pc.b) * p.Hq + pc.hq) * p.Nq + row] =
+            (l_tot > 0.f) ? (m_tot + log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
+      }
+      if (mt == 0) p.ws_ctr[pc.slot] = 0;  // every piece has arrived: ready for the next launch
+    }
+   }
   }
 
   // ---- teardown: all TMEM traffic is finished before the columns are freed ----
@@ -595,7 +1026,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // One warp waits on an mbarrier nothing arrives on; the bounded wait runs out.
-__global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
+__global__ void selftest_timeout_kernel(uint32_t limit_ns) {
   __shared__ __align__(8) uint64_t bar_storage;
   __shared__ int abort_storage;
   if (threadIdx.x == 0) {
@@ -604,7 +1035,7 @@ __global__ void selftest_timeout_kernel(unsigned long long limit_ns) {
     fence_mbar_init();
   }
   __syncwarp();
-  const WaitGuard g{&abort_storage, &g_status, limit_ns};
+  const WaitGuard g{smem_addr(&abort_storage), limit_ns};
   mbar_wait(smem_addr(&bar_storage), 0, g, FA2_SITE_SELFTEST, 0);
   __syncwarp();
   if (threadIdx.x == 0) mbar_arrive(smem_addr(&bar_storage));  // leave the barrier consistent
@@ -658,12 +1089,57 @@ static int validate_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
   if (q_bytes >= lim || kv_bytes >= lim) return FA2_ERR_SIZE;
   const long long nblk = (static_cast<long long>(Nq) + kRowsPerCta - 1) / kRowsPerCta;
   if (nblk * Hq * B > INT_MAX) return FA2_ERR_SIZE;
+  // one round of units (all heads and batches of a query block) must count
+  // fewer than 2^31 K/V-tile iterations
+  const long long nkt = (static_cast<long long>(Nk) + kBlockN - 1) / kBlockN;
+  if (nkt * Hq * B >= (1LL << 31)) return FA2_ERR_SIZE;
   return FA2_OK;
+}
+
+// Host-side plan of the work decomposition (same unit order and sizes as the
+// device iterator).
+struct Plan {
+  int n_qblk = 0;
+  long long units = 0;  // (query block, head, batch) units
+  long long iters = 0;  // K/V-tile iterations summed over all units
+  long long T = 0;      // summed unit costs (kUnitCost + iterations per non-empty unit)
+  int G = 0;            // stream-K CTAs (0 when there is nothing to compute)
+  long long ws_bytes = 0;
+};
+
+constexpr long long kCtrBytes = 256;  // alignment of the partials after the counters
+
+static Plan make_plan(int B, int Hq, int Nq, int Nk, int causal, int d, int num_sms) {
+  Plan pl;
+  pl.n_qblk = (Nq + kRowsPerCta - 1) / kRowsPerCta;
+  const long long HB = static_cast<long long>(B) * Hq;
+  pl.units = HB * pl.n_qblk;
+  for (int qb = 0; qb < pl.n_qblk; ++qb) {
+    const int n = unit_tiles(Nq, Nk, causal, qb);
+    pl.iters += HB * n;
+    pl.T += HB * (n > 0 ? n + kUnitCost : 0);
+  }
+  if (pl.iters == 0 || num_sms <= 0) return pl;
+  pl.G = static_cast<int>(pl.iters < num_sms ? pl.iters : num_sms);
+  // a CTA's range holds at most two pieces of split units (its first and its
+  // last), so two partial buffers per CTA cover every split
+  const long long piece_bytes = 4LL * kTiles * kBlockM * (d + 2);
+  const long long ctr = ((4LL * pl.G + kCtrBytes - 1) / kCtrBytes) * kCtrBytes;
+  pl.ws_bytes = (pl.G > 1) ? ctr + 2LL * pl.G * piece_bytes : 0;
+  return pl;
+}
+
+static int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
 }
 
 template <int D>
 static int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                  int Hkv, int Nq, int Nk, int causal, float scale, cudaStream_t stream) {
+                  int Hkv, int Nq, int Nk, int causal, float scale, void* workspace,
+                  long long workspace_bytes, cudaStream_t stream) {
   using C = Cfg<D>;
   static std::once_flag once;
   static int setup_status = FA2_OK;
@@ -683,11 +1159,6 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
   });
   if (setup_status != FA2_OK) return setup_status;
 
-  CUtensorMap tq, tk, tv;
-  if (!encode_bnhd(&tq, q, B, Nq, Hq, D) || !encode_bnhd(&tk, k, B, Nk, Hkv, D) ||
-      !encode_bnhd(&tv, v, B, Nk, Hkv, D))
-    return FA2_ERR_LAUNCH;
-
   Params p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -703,8 +1174,36 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
   // c * (s - m) ~ 1e-30 * O(1e4), which rounds to exp2(0) = 1 as required.
   p.c = std::fmax(std::fabs(scale) * 1.4426950408889634f, 1e-30f);
   p.negate = scale < 0.f ? 1 : 0;
-  p.limit_ns = 1000000000ull;  // 1 s per wait; a healthy wait takes microseconds
-  const unsigned grid = static_cast<unsigned>(p.n_qblk) * Hq * B;
+  p.limit_ns = 1000000000u;  // 1 s per wait; a healthy wait takes microseconds
+  p.streamk = 0;
+  p.T = 0;
+  p.span = 0;
+  p.rem = 0;
+  p.G = 1;
+  p.ws = nullptr;
+  p.ws_ctr = nullptr;
+  unsigned grid = static_cast<unsigned>(p.n_qblk) * Hq * B;  // one unit per CTA
+  if (workspace) {
+    const Plan pl = make_plan(B, Hq, Nq, Nk, p.causal, D, sm_count());
+    if (pl.G > 0) {  // otherwise every unit is empty: one CTA per unit writes it
+      if (pl.T > INT_MAX) return FA2_ERR_SIZE;
+      if (workspace_bytes < pl.ws_bytes) return FA2_ERR_WORKSPACE;
+      p.streamk = 1;
+      p.T = static_cast<int>(pl.T);
+      p.G = pl.G;
+      p.span = static_cast<int>(pl.T / pl.G);
+      p.rem = static_cast<int>(pl.T % pl.G);
+      p.ws_ctr = static_cast<int*>(workspace);
+      const long long ctr = ((4LL * pl.G + kCtrBytes - 1) / kCtrBytes) * kCtrBytes;
+      p.ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + ctr);
+      grid = static_cast<unsigned>(pl.G);
+    }
+  }
+
+  CUtensorMap tq, tk, tv;
+  if (!encode_bnhd(&tq, q, B, Nq, Hq, D) || !encode_bnhd(&tk, k, B, Nk, Hkv, D) ||
+      !encode_bnhd(&tv, v, B, Nk, Hkv, D))
+    return FA2_ERR_LAUNCH;
   fa2_fwd_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_LAUNCH;
 }
@@ -728,22 +1227,65 @@ static int check_device() {
 
 using namespace fa2;
 
-extern "C" int fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                           int Hq, int Hkv, int Nq, int Nk, int d, int causal, float softmax_scale,
-                           void* stream) {
+static int forward_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int Nq, int Nk, int d, int causal, float softmax_scale,
+                        void* workspace, long long workspace_bytes, void* stream) {
   if (!q || !k || !v || !o || !lse) return FA2_ERR_NULL_POINTER;
   const int sv = validate_shape(B, Hq, Hkv, Nq, Nk, d);
   if (sv != FA2_OK) return sv;
   if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
-       reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o)) & 15u)
+       reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o) |
+       reinterpret_cast<uintptr_t>(workspace)) & 15u)
     return FA2_ERR_ALIGNMENT;
   if (reinterpret_cast<uintptr_t>(lse) & 3u) return FA2_ERR_ALIGNMENT;
   if (!std::isfinite(softmax_scale)) return FA2_ERR_SCALE;
+  if (workspace && workspace_bytes < 0) return FA2_ERR_WORKSPACE;
   const int dv = check_device();
   if (dv != FA2_OK) return dv;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 128) return launch<128>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal, softmax_scale, s);
-  return launch<64>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal, softmax_scale, s);
+  if (d == 128)
+    return launch<128>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal, softmax_scale, workspace,
+                       workspace_bytes, s);
+  return launch<64>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal, softmax_scale, workspace,
+                    workspace_bytes, s);
+}
+
+extern "C" int fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                           int Hq, int Hkv, int Nq, int Nk, int d, int causal, float softmax_scale,
+                           void* stream) {
+  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, nullptr, 0,
+                      stream);
+}
+
+extern "C" int fa2_forward_ws(const void* q, const void* k, const void* v, void* o, float* lse,
+                              int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                              float softmax_scale, void* workspace, long long workspace_bytes,
+                              void* stream) {
+  if (!workspace) return FA2_ERR_NULL_POINTER;
+  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, workspace,
+                      workspace_bytes, stream);
+}
+
+extern "C" long long fa2_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal) {
+  if (validate_shape(B, Hq, Hkv, Nq, Nk, d) != FA2_OK) return -1;
+  const int n = sm_count();
+  if (n <= 0) return -1;
+  const Plan pl = make_plan(B, Hq, Nq, Nk, causal ? 1 : 0, d, n);
+  return pl.T > INT_MAX ? -1 : pl.ws_bytes;
+}
+
+extern "C" int fa2_streamk_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                                int num_sms, long long* total_iters, int* ctas,
+                                long long* workspace_bytes) {
+  const int sv = validate_shape(B, Hq, Hkv, Nq, Nk, d);
+  if (sv != FA2_OK) return sv;
+  if (num_sms <= 0) return FA2_ERR_BAD_SHAPE;
+  const Plan pl = make_plan(B, Hq, Nq, Nk, causal ? 1 : 0, d, num_sms);
+  if (pl.T > INT_MAX) return FA2_ERR_SIZE;
+  if (total_iters) *total_iters = pl.iters;
+  if (ctas) *ctas = pl.G;
+  if (workspace_bytes) *workspace_bytes = pl.ws_bytes;
+  return FA2_OK;
 }
 
 extern "C" const char* fa2_status_string(int status) {
@@ -758,6 +1300,7 @@ extern "C" const char* fa2_status_string(int status) {
     case FA2_ERR_LAUNCH: return "CUDA call or kernel launch failed";
     case FA2_ERR_SIZE: return "problem exceeds the supported tensor or grid extent";
     case FA2_ERR_BUILD: return "kernel image does not match its register plan";
+    case FA2_ERR_WORKSPACE: return "workspace smaller than fa2_workspace_size reports";
     default: return "unknown status";
   }
 }
@@ -778,11 +1321,11 @@ extern "C" int fa2_debug_status(void* stream) {
 }
 
 extern "C" int fa2_selftest_timeout(void* stream, long long limit_ns) {
-  if (limit_ns < 1000000LL || limit_ns > 10000000000LL) return FA2_ERR_SIZE;
+  if (limit_ns < 1000000LL || limit_ns > 4000000000LL) return FA2_ERR_SIZE;
   const int dv = check_device();
   if (dv != FA2_OK) return dv;
   selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<unsigned long long>(limit_ns));
+      static_cast<uint32_t>(limit_ns));
   return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_LAUNCH;
 }
 

@@ -114,12 +114,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Where a bounded wait reports a timeout.
+// Status word a bounded wait writes when it gives up: (site << 16) | iteration.
+// The first failure wins.  (One definition: this header is compiled into one
+// translation unit of the library.)
+__device__ int g_status = 0;
+
+// How a bounded wait may give up.
 struct WaitGuard {
-  volatile int* abort_flag;     // shared-memory flag: set once anything in the CTA gave up
-  int* status;                  // global status word (first failure wins)
-  unsigned long long limit_ns;  // time limit per wait
+  uint32_t abort_smem;          // shared-memory address of the CTA's abort flag; 0 = ignore it
+  uint32_t limit_ns;            // time limit per wait (below 2^32 ns, about 4.29 s)
 };
+
+__device__ __forceinline__ int ld_volatile_shared(uint32_t addr) {
+  int v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_volatile_shared(uint32_t addr, int v) {
+  asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 
 // Wait until the phase with the given parity of `bar` has completed.  Returns
 // false (after recording `site`/`iter` in the status word and raising the CTA's
@@ -131,11 +144,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   for (uint32_t spin = 1;; ++spin) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((spin & 31u) == 0) {
-      if (*g.abort_flag) return false;
+      if (g.abort_smem && ld_volatile_shared(g.abort_smem)) return false;
       if (global_timer_ns() - t0 > g.limit_ns) {
-        const int code = (site << 16) | (iter & 0xffff);
-        atomicCAS(g.status, 0, code);
-        *g.abort_flag = 1;
+        atomicCAS(&g_status, 0, (site << 16) | (iter & 0xffff));
+        if (g.abort_smem) st_volatile_shared(g.abort_smem, 1);
         __threadfence_block();
         return false;
       }
@@ -210,6 +222,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
+}
+
+// Each thread of a warp reads 8 consecutive 32-bit columns of its own lane.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
 }
 
 // Each thread of a warp reads 16 consecutive 32-bit columns of its own lane.

@@ -24,7 +24,8 @@
  *   - a row with no visible key gets O = 0 and LSE = -inf;
  *   - LSE is the natural log and includes softmax_scale.
  *
- * All entry points are thread-safe and allocate no device memory.
+ * All entry points are thread-safe and allocate no device memory; the
+ * stream-K variant takes its scratch memory from the caller.
  */
 #ifndef FA2_H
 #define FA2_H
@@ -44,7 +45,8 @@ enum fa2_status_code {
   FA2_ERR_DEVICE = 6,         /* current device is not compute capability 10.0      */
   FA2_ERR_LAUNCH = 7,         /* a CUDA runtime/driver call or the launch failed    */
   FA2_ERR_SIZE = 8,           /* a tensor or the grid exceeds the supported extent   */
-  FA2_ERR_BUILD = 9           /* the kernel image does not match its register plan  */
+  FA2_ERR_BUILD = 9,          /* the kernel image does not match its register plan  */
+  FA2_ERR_WORKSPACE = 10      /* workspace smaller than fa2_workspace_size reports   */
 };
 
 /*
@@ -73,6 +75,60 @@ enum fa2_status_code {
 int fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                 int Hkv, int Nq, int Nk, int d, int causal, float softmax_scale, void* stream);
 
+/*
+ * fa2_forward_ws -- the same computation as fa2_forward, scheduled stream-K
+ * over a caller-provided workspace.
+ *
+ * Units of work are (256-row query block, query head, batch); a unit costs one
+ * iteration per K/V tile it visits.  fa2_forward launches one thread block per
+ * unit, so the last wave of blocks and the longest causal unit leave SMs idle
+ * (the occupancy problem of "FlashAttention 2: Three Places the Chip Was Still
+ * Waiting", section 2.3, and "FlashAttention-2 and -3: From Algebra to GPU
+ * Scheduling", "Why more parallelism has limits").  fa2_forward_ws instead
+ * launches one persistent block per SM and cuts the concatenated iterations of
+ * all units (heaviest first) into equal contiguous ranges, one per block.  A
+ * unit cut by a range boundary is computed in pieces over disjoint K/V
+ * ranges; each piece keeps its own row max m and denominator l, and the last
+ * piece to finish merges them with the identity that makes the softmax
+ * statistics mergeable (m = max m_i, l = sum l_i e^(m_i - m),
+ * O = sum O_i e^(m_i - m) / l): the same page, "Keep the unchanged
+ * mathematical target in view" and "Another use of mergeable statistics".
+ * Partials are kept in fp32, so the result equals fa2_forward's up to the
+ * order of floating-point rounding.
+ *
+ *   workspace        device pointer, 16-byte aligned, at least
+ *                    fa2_workspace_size(...) bytes for this problem on the
+ *                    current device.  Its first fa2_workspace_size counters
+ *                    (4 bytes per SM, rounded up to 256 bytes) must be zero
+ *                    before the first call; every completed call leaves them
+ *                    zero again, so one zero-fill at allocation suffices.
+ *                    The rest is scratch the call overwrites.
+ *   workspace_bytes  size of `workspace` in bytes
+ *   (other arguments as in fa2_forward)
+ *
+ * Returns FA2_ERR_NULL_POINTER for a NULL workspace, FA2_ERR_WORKSPACE
+ * when workspace_bytes is smaller than required, and FA2_ERR_SIZE when the
+ * problem has 2^31 or more K/V-tile iterations in total (far beyond any
+ * single call worth scheduling this way; fa2_forward has no such limit).  Calls that may run at the
+ * same time (different streams without ordering between them) need separate
+ * workspaces; calls ordered on one stream may share one.  A call that gave up
+ * on a wait (see fa2_debug_status) may leave counters nonzero: zero the
+ * workspace again before reusing it.
+ */
+int fa2_forward_ws(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                   int Hkv, int Nq, int Nk, int d, int causal, float softmax_scale,
+                   void* workspace, long long workspace_bytes, void* stream);
+
+/*
+ * fa2_workspace_size -- bytes of workspace fa2_forward_ws needs for this
+ * problem on the current device (0 when no unit is split, e.g. one SM's worth
+ * of work).  Returns -1 for an invalid shape (as fa2_forward validates it),
+ * for a problem fa2_forward_ws refuses with FA2_ERR_SIZE, or when the device
+ * cannot be queried.  Queries the device's SM count; makes no
+ * other CUDA call.
+ */
+long long fa2_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal);
+
 /* Human-readable text for a status code (static storage, never NULL). */
 const char* fa2_status_string(int status);
 
@@ -97,12 +153,13 @@ enum fa2_wait_site {
   FA2_SITE_FINAL_STATS = 9,
   FA2_SITE_MMA_DRAIN = 10,
   FA2_SITE_LOAD_DRAIN = 11,
+  FA2_SITE_MERGE = 12,        /* stream-K: partial published / merge job hand-off */
   FA2_SITE_SELFTEST = 15
 };
 
 /*
  * fa2_selftest_timeout -- launch a one-warp kernel that waits on an mbarrier
- * nothing ever arrives on, with the given limit in nanoseconds (1 ms .. 10 s),
+ * nothing ever arrives on, with the given limit in nanoseconds (1 ms .. 4 s),
  * through the same bounded-wait routine the attention kernel uses.  The wait
  * runs out, the kernel records FA2_SITE_SELFTEST and returns; read it with
  * fa2_debug_status.  Exercises the failure path without faulting the GPU.
@@ -124,6 +181,17 @@ int fa2_selftest_timeout(void* stream, long long limit_ns);
 long long fa2_num_blocks(int B, int H, int N, int rows_per_block);
 int fa2_launch_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int* grid_blocks,
                     int* threads_per_block, int* smem_bytes, int* rows_per_block);
+
+/*
+ * fa2_streamk_plan: the stream-K schedule fa2_forward_ws would use on a GPU
+ * with num_sms SMs: total K/V-tile iterations over all units, persistent
+ * blocks launched (min(num_sms, total); 0 when every unit is empty) and the
+ * workspace bytes.  Any output pointer may be NULL.  Returns an
+ * fa2_status_code (validation as in fa2_forward, minus pointers;
+ * FA2_ERR_BAD_SHAPE for num_sms <= 0, FA2_ERR_SIZE as fa2_forward_ws).
+ */
+int fa2_streamk_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, int num_sms,
+                     long long* total_iters, int* ctas, long long* workspace_bytes);
 
 #ifdef __cplusplus
 }

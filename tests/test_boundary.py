@@ -67,7 +67,7 @@ def test_valid_arguments_reach_the_device_check_only():
 
 
 def test_status_strings():
-    for code in range(10):
+    for code in range(11):
         assert isinstance(fa2.fa2_status_string(code), str)
     assert fa2.fa2_status_string(12345) == "unknown status"
 

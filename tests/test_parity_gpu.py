@@ -1,5 +1,10 @@
 """GPU forward pass vs the fp64 oracle, element by element, through the C ABI.
 
+Every case runs under both schedules: one thread block per unit
+(``fa2_forward``) and stream-K over a workspace (``fa2_forward_ws``), which on
+a 148-SM GPU splits the units of every workload here that has more than one
+unit's worth of iterations per SM or fewer units than SMs.
+
 Tolerances (on every compared row): O max-abs <= 2e-2 and mean-abs <= 2e-3,
 LSE max-abs <= 1e-3, no NaN/Inf where the oracle is finite.
 """
@@ -26,9 +31,19 @@ def fa2():
     return m
 
 
-def run_gpu(fa2, q, k, v, causal, scale, guard=0):
+@pytest.fixture(params=["units", "streamk"])
+def sched(request):
+    return request.param
+
+
+def counter_bytes(G):
+    return -(-4 * G // 256) * 256
+
+
+def run_gpu(fa2, q, k, v, causal, scale, guard=0, sched="units"):
     """Run the C-ABI forward on copies of q, k, v; O and LSE are carved out of
-    NaN-filled buffers with `guard` poisoned elements on both sides."""
+    NaN-filled buffers with `guard` poisoned elements on both sides.  Under
+    stream-K the workspace's counters must be back at zero afterwards."""
     dev = torch.device("cuda")
     qd, kd, vd = (t.to(dev).contiguous() for t in (q, k, v))
     B, Nq, Hq, d = q.shape
@@ -39,11 +54,23 @@ def run_gpu(fa2, q, k, v, causal, scale, guard=0):
     gl = max(guard, 4)
     o = o_buf[g_o:g_o + B * Nq * Hq * d].view(B, Nq, Hq, d)
     lse = l_buf[gl:gl + B * Hq * Nq].view(B, Hq, Nq)
-    st = fa2.fa2_forward(qd, kd, vd, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale,
-                         torch.cuda.current_stream())
+    ws = None
+    if sched == "units":
+        st = fa2.fa2_forward(qd, kd, vd, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale,
+                             torch.cuda.current_stream())
+    else:
+        ws = fa2.alloc_workspace(B, Hq, Hkv, Nq, Nk, d, causal, dev)
+        st = fa2.fa2_forward_ws(qd, kd, vd, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, ws,
+                                ws.numel(), torch.cuda.current_stream())
     assert st == 0, fa2.fa2_status_string(st)
     torch.cuda.synchronize()
     assert fa2.fa2_debug_status(None) == 0
+    if ws is not None:
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        _, _, G, wsb = fa2.fa2_streamk_plan(B, Hq, Hkv, Nq, Nk, d, causal, sms)
+        assert wsb <= ws.numel()
+        if wsb:
+            assert int(ws[:counter_bytes(G)].count_nonzero()) == 0, "counters not reset"
     if guard:
         assert torch.isnan(o_buf[:g_o].float()).all() and torch.isnan(o_buf[-g_o:].float()).all(), \
             "O guard band overwritten"
@@ -66,33 +93,33 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
     return float(err.max()), float(err.mean())
 
 
-def check_case(fa2, w: Workload, rows=None, scale=None, guard=0):
+def check_case(fa2, w: Workload, rows=None, scale=None, guard=0, sched="units"):
     q, k, v = make_qkv(w)
     scale = w.softmax_scale if scale is None else scale
-    o_gpu, lse_gpu = run_gpu(fa2, q, k, v, w.causal, scale, guard=guard)
+    o_gpu, lse_gpu = run_gpu(fa2, q, k, v, w.causal, scale, guard=guard, sched=sched)
     o_ref, lse_ref = oracle.attention(bf16_bits(q), bf16_bits(k), bf16_bits(v), w.causal, scale,
                                       rows=rows)
     if rows is not None:
         o_gpu, lse_gpu = o_gpu[:, rows], lse_gpu[:, :, rows]
-    return compare(o_gpu, lse_gpu, o_ref, lse_ref, what=w.name)
+    return compare(o_gpu, lse_gpu, o_ref, lse_ref, what=f"{w.name}/{sched}")
 
 
 # ---- the five specified workloads, in the launch configuration the benchmark times ----
 
-def test_tiny_all_rows(fa2):
-    check_case(fa2, WORKLOADS["tiny"], guard=8)
+def test_tiny_all_rows(fa2, sched):
+    check_case(fa2, WORKLOADS["tiny"], guard=8, sched=sched)
 
 
-def test_noncausal_2k_all_rows(fa2):
-    check_case(fa2, WORKLOADS["noncausal_2k"])
+def test_noncausal_2k_all_rows(fa2, sched):
+    check_case(fa2, WORKLOADS["noncausal_2k"], sched=sched)
 
 
 @pytest.mark.parametrize("name", ["causal_8k", "long_32k", "gqa_4k"])
-def test_full_size_sampled_rows(fa2, name):
+def test_full_size_sampled_rows(fa2, name, sched):
     w = WORKLOADS[name]
     idx = list(WORKLOADS).index(name)
     rows = sample_rows(w, 1024, seed=idx)
-    check_case(fa2, w, rows=rows)
+    check_case(fa2, w, rows=rows, sched=sched)
 
 
 # ---- ragged and odd sizes, both head dims, Nq != Nk in both directions ----
@@ -104,28 +131,43 @@ ODD = [1, 17, 127, 129, 1000]
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("nq,nk", [(n, n) for n in ODD] + [(17, 1000), (1000, 17), (129, 127),
                                                             (127, 129), (1, 1000), (300, 1)])
-def test_odd_sizes(fa2, d, causal, nq, nk):
+def test_odd_sizes(fa2, d, causal, nq, nk, sched):
     w = Workload(f"odd{nq}x{nk}", 2, 4, 2, nq, nk, d, causal, seed=nq * 7 + nk)
-    check_case(fa2, w, guard=8)
+    check_case(fa2, w, guard=8, sched=sched)
 
 
 @pytest.mark.parametrize("scale", [0.0, -0.0883883, 0.5])
-def test_scale_values(fa2, scale):
+def test_scale_values(fa2, scale, sched):
     w = Workload("scale", 1, 2, 1, 300, 300, 128, True, seed=3)
-    check_case(fa2, w, scale=scale)
+    check_case(fa2, w, scale=scale, sched=sched)
 
 
-def test_large_scores_outliers_d64(fa2):
+def test_large_scores_outliers_d64(fa2, sched):
     w = Workload("outl64", 1, 2, 2, 2048, 2048, 64, True, seed=5, outlier_frac=0.01, outlier_scale=8.0)
-    check_case(fa2, w)
+    check_case(fa2, w, sched=sched)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_one_long_unit_cut_into_many_pieces(fa2, d, sched):
+    # one query block against 64k keys: stream-K cuts the single unit at every
+    # SM's range boundary and merges ~148 partials
+    w = Workload("longkv", 1, 1, 1, 256, 65536, d, False, seed=21)
+    check_case(fa2, w, sched=sched)
+
+
+def test_causal_more_queries_than_keys_streamk_rows(fa2, sched):
+    # Nq > Nk causal: leading query blocks see no key (empty units written
+    # outside the stream-K ranges) while the rest are split
+    w = Workload("nq>nk", 2, 3, 1, 3000, 1100, 128, True, seed=22)
+    check_case(fa2, w, guard=8, sched=sched)
 
 
 # ---- closed forms on the GPU ----
 
-def test_causal_row0_is_v0_bitwise(fa2):
+def test_causal_row0_is_v0_bitwise(fa2, sched):
     w = Workload("row0", 2, 4, 2, 384, 384, 128, True, seed=9)
     q, k, v = make_qkv(w)
-    o, lse = run_gpu(fa2, q, k, v, True, w.softmax_scale)
+    o, lse = run_gpu(fa2, q, k, v, True, w.softmax_scale, sched=sched)
     vv = v.float().numpy()
     for hq in range(4):
         assert np.array_equal(o[:, 0, hq], vv[:, 0, hq // 2]), "row 0 must be exactly V[0]"
@@ -133,11 +175,11 @@ def test_causal_row0_is_v0_bitwise(fa2):
     assert np.abs(lse[:, :, 0] - w.softmax_scale * qk).max() < 1e-3
 
 
-def test_zero_query_gives_mean_of_visible_v(fa2):
+def test_zero_query_gives_mean_of_visible_v(fa2, sched):
     w = Workload("q0", 1, 2, 2, 260, 260, 64, True, seed=10)
     q, k, v = make_qkv(w)
     q = torch.zeros_like(q)
-    o, lse = run_gpu(fa2, q, k, v, True, w.softmax_scale)
+    o, lse = run_gpu(fa2, q, k, v, True, w.softmax_scale, sched=sched)
     vv = v.double().numpy()
     csum = np.cumsum(vv, axis=1) / np.arange(1, 261)[None, :, None, None]
     assert np.abs(o - csum).max() < 2e-2
@@ -146,19 +188,21 @@ def test_zero_query_gives_mean_of_visible_v(fa2):
 
 # ---- structural properties ----
 
-def test_gqa_equals_repeated_heads_bitwise(fa2):
+def test_gqa_equals_repeated_heads_bitwise(fa2, sched):
     w = Workload("gqa", 2, 8, 2, 700, 700, 128, True, seed=12)
     q, k, v = make_qkv(w)
-    o1, l1 = run_gpu(fa2, q, k, v, True, w.softmax_scale)
+    o1, l1 = run_gpu(fa2, q, k, v, True, w.softmax_scale, sched=sched)
     o2, l2 = run_gpu(fa2, q, k.repeat_interleave(4, dim=2), v.repeat_interleave(4, dim=2), True,
-                     w.softmax_scale)
+                     w.softmax_scale, sched=sched)
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
 
 
-def test_deterministic_across_runs(fa2):
+def test_deterministic_across_runs(fa2, sched):
+    # stream-K merges the pieces of a split unit in their order in the unit,
+    # whichever CTA finishes last, so it is deterministic too
     w = Workload("det", 2, 4, 4, 1500, 1500, 128, True, seed=13)
     q, k, v = make_qkv(w)
-    outs = [run_gpu(fa2, q, k, v, True, w.softmax_scale) for _ in range(3)]
+    outs = [run_gpu(fa2, q, k, v, True, w.softmax_scale, sched=sched) for _ in range(3)]
     for o, l in outs[1:]:
         assert np.array_equal(o, outs[0][0]) and np.array_equal(l, outs[0][1])
 
@@ -170,3 +214,50 @@ def test_torch_convenience_wrapper(fa2):
     torch.cuda.synchronize()
     o_ref, l_ref = oracle.attention(bf16_bits(q), bf16_bits(k), bf16_bits(v), False, w.softmax_scale)
     compare(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, what="wrapper")
+
+
+def test_streamk_matches_units_closely(fa2):
+    # same arithmetic per key tile; only the split units' merge rounds differently
+    w = Workload("sk_vs_u", 2, 16, 16, 4096, 4096, 128, True, seed=23)
+    q, k, v = make_qkv(w)
+    o1, l1 = run_gpu(fa2, q, k, v, True, w.softmax_scale, sched="units")
+    o2, l2 = run_gpu(fa2, q, k, v, True, w.softmax_scale, sched="streamk")
+    assert np.abs(o1 - o2).max() <= 1.6e-2
+    assert np.abs(l1 - l2).max() <= 1e-4
+
+
+def test_workspace_reused_across_calls_and_shapes(fa2):
+    # one zero-filled workspace, sized for the largest problem, serves calls of
+    # different shapes ordered on one stream
+    dev = torch.device("cuda")
+    shapes = [Workload("r1", 2, 16, 16, 4096, 4096, 128, True, seed=24),
+              Workload("r2", 1, 4, 2, 1000, 3000, 64, False, seed=25),
+              Workload("r3", 2, 16, 16, 4096, 4096, 128, True, seed=24)]
+    need = max(fa2.fa2_workspace_size(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal) for w in shapes)
+    ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+    outs = []
+    for w in shapes:
+        q, k, v = (t.to(dev) for t in make_qkv(w))
+        o, lse = fa2.attention(q, k, v, causal=w.causal, workspace=ws)
+        outs.append((o.float().cpu().numpy(), lse.cpu().numpy()))
+    torch.cuda.synchronize()
+    assert fa2.fa2_debug_status(None) == 0
+    assert np.array_equal(outs[0][0], outs[2][0]) and np.array_equal(outs[0][1], outs[2][1])
+    w = shapes[1]
+    q, k, v = make_qkv(w)
+    o_ref, l_ref = oracle.attention(bf16_bits(q), bf16_bits(k), bf16_bits(v), w.causal, w.softmax_scale)
+    compare(outs[1][0], outs[1][1], o_ref, l_ref, what="reused workspace")
+
+
+def test_small_workspace_is_refused(fa2):
+    w = Workload("small_ws", 2, 16, 16, 4096, 4096, 128, True, seed=26)
+    dev = torch.device("cuda")
+    need = fa2.fa2_workspace_size(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal)
+    assert need > 0
+    q, k, v = (t.to(dev) for t in make_qkv(w))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    ws = torch.zeros(need - 256, dtype=torch.uint8, device=dev)
+    st = fa2.fa2_forward_ws(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
+                            w.softmax_scale, ws, ws.numel(), torch.cuda.current_stream())
+    assert st == 10

@@ -23,7 +23,7 @@ STATUS_NAMES = {
 SITE_NAMES = {
     1: "Q_LOADED", 2: "KV_LOADED", 3: "KV_FREE", 4: "S_READY", 5: "P_READY", 6: "STATS_READY",
     7: "O_RESCALED", 8: "O_FINAL", 9: "FINAL_STATS", 10: "MMA_DRAIN", 11: "LOAD_DRAIN",
-    12: "MERGE", 15: "SELFTEST",
+    15: "SELFTEST",
 }
 FA2_SITE_SELFTEST = 15
 
@@ -141,17 +141,14 @@ def fa2_launch_plan(B, Hq, Hkv, Nq, Nk, d):
 # ---- torch convenience: allocate outputs with torch, then call the C ABI ----
 
 def alloc_workspace(B, Hq, Hkv, Nq, Nk, d, causal, device):
-    """A zero-filled uint8 CUDA tensor large enough for ``fa2_forward_ws``.
-
-    Zero once here; every completed call leaves the counters zero again, so
-    the tensor can be reused by later calls ordered on the same stream.
-    """
+    """A uint8 CUDA tensor large enough for ``fa2_forward_ws`` (scratch: no
+    initialisation needed; reusable by later calls ordered on one stream)."""
     import torch
 
     n = fa2_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal)
     if n < 0:
         raise FA2Error(2, "fa2_workspace_size")
-    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
 
 
 def attention(q, k, v, causal: bool = False, softmax_scale: float | None = None, out=None,

@@ -49,11 +49,11 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kSwizzleBytes = 128;  // one swizzle atom row: 64 bf16
 constexpr int kChunkBytes = kBlockM * kSwizzleBytes;  // 64 columns of a 128-row tile
 
-// Register split (per thread): 2 softmax warpgroups x 184 + correction/epilogue
-// 64 + MMA/load warpgroup 80 = 512 = 4 x 128, i.e. exactly the launch pool.
+// Register split (per thread): 2 softmax warpgroups x 192 + correction/epilogue
+// 48 + MMA/load warpgroup 80 = 512 = 4 x 128, i.e. exactly the launch pool.
 // Each role compiles without spills in its budget.
-constexpr int kRegsSoftmax = 184;
-constexpr int kRegsCorrection = 64;
+constexpr int kRegsSoftmax = 192;
+constexpr int kRegsCorrection = 48;
 constexpr int kRegsOther = 80;
 static_assert(2 * kRegsSoftmax + kRegsCorrection + kRegsOther == 4 * kLaunchRegs,
               "register split must equal the launch allocation");
@@ -68,10 +68,7 @@ enum Bar {
   BAR_FSTATS = 10,   // [2] final row max / denominator of a piece published (128 softmax threads)
   BAR_FCONS = 12,    // [2] final statistics read by the epilogue (128 correction threads)
   BAR_DONE = 14,     // all MMAs drained (MMA commit)
-  BAR_GRP = 15,      // a split piece's partial is fully published (128 correction threads)
-  BAR_MJOB = 16,     // merge job posted for a split piece (one correction thread)
-  BAR_MFREE = 17,    // merge job slot read (64 merge threads)
-  BAR_KV_FULL = 18,  // [stages] K/V tile landed (TMA tx); then [stages] slot free (MMA commit)
+  BAR_KV_FULL = 15,  // [stages] K/V tile landed (TMA tx); then [stages] slot free (MMA commit)
 };
 
 // Scheduling cost of a unit, in K/V-tile iterations, on top of its
@@ -81,8 +78,8 @@ enum Bar {
 // fewer iterations.
 constexpr int kUnitCost = 2;
 
-// Warps 14-15 (otherwise idle) merge split units and write empty ones.
-constexpr int kMergeThreads = 64;
+// Warps 14-15 (otherwise idle) write the rows of units with no visible key.
+constexpr int kEmptyThreads = 64;
 
 template <int D>
 struct Cfg {
@@ -120,6 +117,7 @@ struct Params {
   int B, Hq, Hkv, Nq, Nk;
   int causal;
   int n_qblk;
+  int r_empty;        // first round (heaviest first) of units with no visible key; n_qblk if none
   float c;            // |softmax_scale| * log2(e)
   int negate;         // softmax_scale < 0: compute S = -(Q K^T) so c stays >= 0
   uint32_t limit_ns;  // per bounded wait
@@ -130,7 +128,6 @@ struct Params {
   int rem;            // T % G
   int G;              // CTAs of a stream-K launch
   float* ws;          // stream-K partials: [G CTAs][2: first / last piece of its range][piece floats]
-  int* ws_ctr;        // [G] arrival counters, zero before the launch and left zero after it
 };
 
 // Number of K/V tiles a 128-row query tile starting at row r0 visits (0 if it
@@ -206,6 +203,7 @@ __device__ __forceinline__ int first_boundary_above(const Params& p, int y) {
 // order.  The next CTA starts with the same unit's tail, so both pieces of a
 // split unit finish early and its merge overlaps the remaining work instead
 // of landing at the end of the kernel.
+template <bool SK>  // SK: stream-K ranges; otherwise CTA u runs unit u whole
 struct PieceIter {
   int HB, r, n, k_cur;
   int cum, x, x_end;  // cost before round r; the natural walk's range [x, x_end)
@@ -240,7 +238,7 @@ struct PieceIter {
     pc.slot = 0;
     pc.npieces = 1;
     pc.index = 0;
-    if (!p.streamk) return;
+    if constexpr (!SK) return;
     const int s_u = cum + k_cur * cost(n) + kUnitCost;                // position of iteration 0
     const int c_first = first_boundary_above(p, s_u);                // B_c > s_u
     const int c_last = first_boundary_above(p, s_u + n - 1) - 1;     // B_c <= s_u + n - 1
@@ -271,7 +269,7 @@ struct PieceIter {
     r = cum = n = k_cur = 0;
     x = x_end = 0;
     state = 1;
-    if (!p.streamk) return;
+    if constexpr (!SK) return;
     x = range_start(p.span, p.rem, p.G, blockIdx.x);
     x_end = range_start(p.span, p.rem, p.G, blockIdx.x + 1);
     state = 0;
@@ -290,7 +288,7 @@ struct PieceIter {
   }
 
   __device__ __forceinline__ bool next(const Params& p, Piece& pc) {
-    if (!p.streamk) {
+    if constexpr (!SK) {
       if (!state) return false;
       state = 0;
       const int u = blockIdx.x;
@@ -372,7 +370,7 @@ __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& e0, fl
 #endif
 constexpr int kEmuPairs = FA2_EMU_PAIRS;
 
-template <int D>
+template <int D, bool SK>
 __global__ void __launch_bounds__(kThreads, 1)
     fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -388,7 +386,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
-  volatile int* sm_job = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);  // 1: merge the unit
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -400,9 +397,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < BAR_KV_FULL; ++i) {
       uint32_t cnt = 1;
       if ((i >= BAR_STATS && i < BAR_STATS + 2) || (i >= BAR_FSTATS && i < BAR_FSTATS + 2) ||
-          (i >= BAR_FCONS && i < BAR_FCONS + 2) || i == BAR_GRP)
+          (i >= BAR_FCONS && i < BAR_FCONS + 2))
         cnt = kBlockM;
-      if (i == BAR_MFREE) cnt = kMergeThreads;
       if (i >= BAR_P && i < BAR_P + 2) cnt = 2 * kBlockM;
       mbar_init(bar(i), cnt);
     }
@@ -430,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the same sequence of pieces with its own iterator.
   if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-    PieceIter pit;
+    PieceIter<SK> pit;
     pit.init(p);
     Piece pc;
     // =================== softmax: one thread per query row ===================
@@ -552,17 +548,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < 12) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCorrection));
-    PieceIter pit;
+    PieceIter<SK> pit;
     pit.init(p);
     Piece pc;
     // ============== correction (O rescale) and epilogue warps ==============
     const int q4 = warp & 3;
     const int rt = q4 * 32 + lane;
-    const int ct = threadIdx.x - 256;  // 0..127 within the correction warps
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     // parities of the phases consumed so far: bit t = STATS_t, bit 2 + t =
-    // OFINAL_t, bit 4 = FSTATS (one per piece), bit 5 = GRP and bit 6 =
-    // MFREE (one per split piece); bit 7: a merge job was posted before
+    // OFINAL_t, bit 4 = FSTATS (one per piece)
     uint32_t ph = 0;
     bool ok = true;
 
@@ -696,33 +690,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       ph ^= 16u;
-      if (!pc.split) continue;
-
-      // ---- split piece: take a ticket once all 128 rows are published and
-      // hand the outcome to the merge warps (the last piece's CTA merges) ----
-      __threadfence();
-      mbar_arrive(bar(BAR_GRP));
-      if (ct == 0) {
-        if (!mbar_wait(bar(BAR_GRP), (ph >> 5) & 1, g, FA2_SITE_MERGE, 0)) {
-          ok = false;
-        } else {
-          const int ticket = atomicAdd(p.ws_ctr + pc.slot, 1);
-          if ((ph & 128u) && !mbar_wait(bar(BAR_MFREE), (ph >> 6) & 1, g, FA2_SITE_MERGE, 1)) {
-            ok = false;
-          } else {
-            *sm_job = (ticket == pc.npieces - 1) ? 1 : 0;
-            mbar_arrive(bar(BAR_MJOB));
-          }
-        }
-      }
-      if (ph & 128u) ph ^= 64u;  // the MFREE phase the last job completed
-      ph ^= 32u;
-      ph |= 128u;
-      if (warp == 8) ok = __all_sync(0xffffffffu, ok);  // keep the warp converged
     }
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
-    PieceIter pit;
+    PieceIter<SK> pit;
     pit.init(p);
     Piece pc;
    if (warp == 12) {
@@ -811,7 +782,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             FA2_SITE_KV_LOADED, pc.jb))
           break;
         tc_fence_after();
-        const uint32_t qfree0 = (n_p == 1) ? bar(BAR_QFREE) : 0u;
+        // (one piece per CTA in unit mode: the Q buffer is never reloaded)
+        const uint32_t qfree0 = (SK && n_p == 1) ? bar(BAR_QFREE) : 0u;
         if (a0 > 0) issue_s(0, itK(0), bar(BAR_S + 0), a1 > 0 ? 0u : free_of(itK(0)), a1 > 0 ? 0u : qfree0);
         if (a1 > 0) issue_s(1, itK(0), bar(BAR_S + 1), free_of(itK(0)), qfree0);
         for (int jj = 0; jj < n_p && ok; ++jj) {
@@ -825,7 +797,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       FA2_SITE_KV_LOADED, pc.jb + jj + 1))
             break;
           // the last S of the piece frees the Q buffer for the next piece
-          const uint32_t qfree = (jj + 2 == n_p) ? bar(BAR_QFREE) : 0u;
+          const uint32_t qfree = (SK && jj + 2 == n_p) ? bar(BAR_QFREE) : 0u;
           // tile 0: PV0(j) and S0(j+1); V_j / K_{j+1} are freed here when tile 1 has no use for them
           if (jj < a0) {
             if (!mbar_wait_warp(bar(BAR_P + 0), p_cnt[0] & 1, g, FA2_SITE_P_READY, pc.jb + jj)) break;
@@ -915,103 +887,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
    } else {
-    // ===================== merge warps (14-15, 64 threads) =====================
-    const int mt = threadIdx.x - (kThreads - kMergeThreads);  // 0..63
+    // ============== warps 14-15: rows of units with no visible key ==============
     // Units with no K/V tile at all (causal, Nq > Nk): O = 0, LSE = -inf.
-    // They form a suffix of the unit order; CTAs share them round robin.
-    {
-      const int HB = p.B * p.Hq;
-      int r0 = 0;  // first round of empty units
-      while (r0 < p.n_qblk && unit_tiles(p.Nq, p.Nk, p.causal, p.n_qblk - 1 - r0) > 0) ++r0;
-      const int nz = (p.n_qblk - r0) * HB;
-      const int z0 = p.streamk ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x) - r0 * HB;
-      const int dz = p.streamk ? p.G : nz;  // unit mode: CTA u owns unit u only
-      for (int z = z0; z >= 0 && z < nz; z += dz) {
-        const int rr = r0 + z / HB, k = z % HB, qb = p.n_qblk - 1 - rr;
-        const int b = k / p.Hq, hq = k % p.Hq;
-        for (int i = mt; i < kRowsPerCta * (D / 8); i += kMergeThreads) {
-          const int row = qb * kRowsPerCta + i / (D / 8);
-          if (row >= p.Nq) continue;
-          reinterpret_cast<uint4*>(p.o + ((static_cast<size_t>(b) * p.Nq + row) * p.Hq + hq) * D)[i % (D / 8)] =
-              make_uint4(0u, 0u, 0u, 0u);
-          if (i % (D / 8) == 0) p.lse[(static_cast<size_t>(b) * p.Hq + hq) * p.Nq + row] = -INFINITY;
-        }
-      }
-    }
-    // Split units: for each split piece of this CTA the correction warps post
-    // whether it was the unit's last piece to publish; if so, merge all its
-    // partials (mergeable statistics: m = max m_i, l = sum l_i 2^(m_i - m),
-    // O = sum O_i 2^(m_i - m) / l), summing in piece order so the result does
-    // not depend on which CTA finished last.
-    uint32_t jobs = 0;
-    bool ok = true;
-    while (ok && pit.next(p, pc)) {
-      pit.split_info(p, pc);
-      if (!pc.split) continue;
-      if (!mbar_wait_warp(bar(BAR_MJOB), jobs & 1, g, FA2_SITE_MERGE, 2)) {
-        ok = false;
-        break;
-      }
-      const bool last = *sm_job != 0;
-      mbar_arrive(bar(BAR_MFREE));
-      ++jobs;
-      if (!last) continue;
-      __threadfence();
-      pit.coords(p, pc);
-      const float* ws = p.ws;
-      asm volatile("" : "+l"(ws));  // keep the address arithmetic here, out of the piece loop
-      auto part = [&](int q) {
-        return ws + static_cast<size_t>(2 * (pc.slot + q) + (q == 0 ? 1 : 0)) * C::kPieceFloats;
-      };
-#pragma unroll 1
-      for (int rr = mt; rr < kRowsPerCta; rr += kMergeThreads) {
-        const int t = rr / kBlockM, rt = rr % kBlockM;
-        const int row = pc.qb * kRowsPerCta + rr;
-        float m_tot = -INFINITY;
-#pragma unroll 1
-        for (int q = 0; q < pc.npieces; ++q)
-          if (__ldcg(part(q) + C::part_l(t, rt)) > 0.f) m_tot = fmaxf(m_tot, __ldcg(part(q) + C::part_m(t, rt)));
-        float l_tot = 0.f;
-#pragma unroll 1
-        for (int q = 0; q < pc.npieces; ++q) {
-          const float lq = __ldcg(part(q) + C::part_l(t, rt));
-          if (lq > 0.f) l_tot = fmaf(lq, ex2_approx(__ldcg(part(q) + C::part_m(t, rt)) - m_tot), l_tot);
-        }
+    // They form a suffix of the unit order; stream-K CTAs share them round robin.
+    const int et = threadIdx.x - (kThreads - kEmptyThreads);  // 0..63
+    const int HB = p.B * p.Hq;
+    const int r0 = p.r_empty;
+    const int nz = (p.n_qblk - r0) * HB;
+    const int z0 = SK ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x) - r0 * HB;
+    const int dz = SK ? p.G : nz;  // unit mode: CTA u owns unit u only
+    for (int z = z0; z >= 0 && z < nz; z += dz) {
+      const int rr = r0 + z / HB, k = z % HB, qb = p.n_qblk - 1 - rr;
+      const int b = k / p.Hq, hq = k % p.Hq;
+      for (int i = et; i < kRowsPerCta * (D / 8); i += kEmptyThreads) {
+        const int row = qb * kRowsPerCta + i / (D / 8);
         if (row >= p.Nq) continue;
-        const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
-        __nv_bfloat16* orow = p.o + ((static_cast<size_t>(pc.b) * p.Nq + row) * p.Hq + pc.hq) * D;
-#pragma unroll 1
-        for (int h = 0; h < D / 8; ++h) {  // 8 columns (half a stored chunk) at a time
-          float acc[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll 1
-          for (int q = 0; q < pc.npieces; ++q) {
-            const float lq = __ldcg(part(q) + C::part_l(t, rt));
-            if (!(lq > 0.f)) continue;
-            const float wq = ex2_approx(__ldcg(part(q) + C::part_m(t, rt)) - m_tot);
-            const float4* src = reinterpret_cast<const float4*>(part(q) + C::part_o(t, h >> 1, rt) + 8 * (h & 1));
-            const float4 f0 = __ldcg(src), f1 = __ldcg(src + 1);
-            acc[0] = fmaf(wq, f0.x, acc[0]);
-            acc[1] = fmaf(wq, f0.y, acc[1]);
-            acc[2] = fmaf(wq, f0.z, acc[2]);
-            acc[3] = fmaf(wq, f0.w, acc[3]);
-            acc[4] = fmaf(wq, f1.x, acc[4]);
-            acc[5] = fmaf(wq, f1.y, acc[5]);
-            acc[6] = fmaf(wq, f1.z, acc[6]);
-            acc[7] = fmaf(wq, f1.w, acc[7]);
-          }
-          uint4 w;
-          w.x = pack_bf16x2(acc[0] * inv_l, acc[1] * inv_l);
-          w.y = pack_bf16x2(acc[2] * inv_l, acc[3] * inv_l);
-          w.z = pack_bf16x2(acc[4] * inv_l, acc[5] * inv_l);
-          w.w = pack_bf16x2(acc[6] * inv_l, acc[7] * inv_l);
-          reinterpret_cast<uint4*>(orow)[h] = w;
-        }
-        p.lse[(static_cast<size_t>(pc.b) * p.Hq + pc.hq) * p.Nq + row] =
-            (l_tot > 0.f) ? (m_tot + log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
+        reinterpret_cast<uint4*>(p.o + ((static_cast<size_t>(b) * p.Nq + row) * p.Hq + hq) * D)[i % (D / 8)] =
+            make_uint4(0u, 0u, 0u, 0u);
+        if (i % (D / 8) == 0) p.lse[(static_cast<size_t>(b) * p.Hq + hq) * p.Nq + row] = -INFINITY;
       }
-      if (mt == 0) p.ws_ctr[pc.slot] = 0;  // every piece has arrived: ready for the next launch
     }
    }
   }
@@ -1023,6 +917,100 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// ---------------------------------------------------------------------------
+// Split-KV merge: after the stream-K kernel, every unit cut by a range boundary
+// has np partials (O unnormalised in fp32, row max m and denominator l over
+// its own K/V range); they combine with the identity that makes the softmax
+// statistics mergeable: m = max m_i, l = sum l_i 2^(m_i - m),
+// O = sum O_i 2^(m_i - m) / l, LSE = (m + log2 l) ln 2 ("FlashAttention-2 and
+// -3: From Algebra to GPU Scheduling", "Keep the unchanged mathematical target
+// in view" and "Another use of mergeable statistics").  Pieces are summed in
+// their order in the unit, so the result is deterministic.
+//
+// Grid: (boundary c = 1..G-1) x (64-row block of the unit's 256 rows) x
+// (16-column chunk of d).  The CTA of boundary c works only if B_c is the
+// first boundary inside some unit's iterations; 4 threads share a row, each
+// owning 4 consecutive columns, so a warp reads 512 contiguous bytes.
+// ---------------------------------------------------------------------------
+constexpr int kCombineThreads = 256;
+constexpr int kCombineRows = 64;
+
+template <int D>
+__global__ void __launch_bounds__(kCombineThreads) fa2_combine_kernel(const Params p) {
+  using C = Cfg<D>;
+  const int c = static_cast<int>(blockIdx.x) + 1;
+  const int bc = range_start(p.span, p.rem, p.G, c);
+  PieceIter<true> it;
+  it.HB = p.B * p.Hq;
+  it.seek_round(p, bc);
+  const int w = PieceIter<true>::cost(it.n);
+  const int k = (bc - it.cum) / w;
+  const int s0 = it.cum + k * w + kUnitCost;  // position of the unit's iteration 0
+  if (!(bc > s0 && bc <= s0 + it.n - 1)) return;                  // B_c cuts no unit
+  if (c > 1 && range_start(p.span, p.rem, p.G, c - 1) > s0) return;  // not the unit's first cut
+  const int np = first_boundary_above(p, s0 + it.n - 1) - c + 1;   // pieces of the unit
+  const int slot = c - 1;                                          // CTA of piece 0
+  const int qb = p.n_qblk - 1 - it.r, b = k / p.Hq, hq = k % p.Hq;
+
+  const int rr = static_cast<int>(blockIdx.y) * kCombineRows + static_cast<int>(threadIdx.x) / 4;
+  const int f4 = threadIdx.x % 4;
+  const int ch = blockIdx.z;
+  const int t = rr / kBlockM, rt = rr % kBlockM;
+  const int row = qb * kRowsPerCta + rr;
+  if (row >= p.Nq) return;
+  auto part = [&](int q) {
+    return p.ws + static_cast<size_t>(2 * (slot + q) + (q == 0 ? 1 : 0)) * C::kPieceFloats;
+  };
+  constexpr int kBatch = 4;  // loads of 4 pieces in flight before any is used
+  float m_tot = -INFINITY;
+  for (int q0 = 0; q0 < np; q0 += kBatch) {
+    float mq[kBatch], lq[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const bool in = q0 + i < np;
+      lq[i] = in ? __ldcg(part(q0 + i) + C::part_l(t, rt)) : 0.f;
+      mq[i] = in ? __ldcg(part(q0 + i) + C::part_m(t, rt)) : -INFINITY;
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i)
+      if (lq[i] > 0.f) m_tot = fmaxf(m_tot, mq[i]);
+  }
+  float l_tot = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int q0 = 0; q0 < np; q0 += kBatch) {
+    float mq[kBatch], lq[kBatch];
+    float4 f[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const bool in = q0 + i < np;
+      const float* base = part(in ? q0 + i : q0);
+      lq[i] = in ? __ldcg(base + C::part_l(t, rt)) : 0.f;
+      mq[i] = __ldcg(base + C::part_m(t, rt));
+      // a piece with l = 0 may not have written its O: loaded, then skipped
+      f[i] = __ldcg(reinterpret_cast<const float4*>(base + C::part_o(t, ch, rt)) + f4);
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      if (!(lq[i] > 0.f)) continue;
+      const float wq = ex2_approx(mq[i] - m_tot);
+      l_tot = fmaf(lq[i], wq, l_tot);
+      acc.x = fmaf(wq, f[i].x, acc.x);
+      acc.y = fmaf(wq, f[i].y, acc.y);
+      acc.z = fmaf(wq, f[i].z, acc.z);
+      acc.w = fmaf(wq, f[i].w, acc.w);
+    }
+  }
+  const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
+  __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Nq + row) * p.Hq + hq) * D;
+  uint2 o2;
+  o2.x = pack_bf16x2(acc.x * inv_l, acc.y * inv_l);
+  o2.y = pack_bf16x2(acc.z * inv_l, acc.w * inv_l);
+  reinterpret_cast<uint2*>(orow + 16 * ch)[f4] = o2;
+  if (ch == 0 && f4 == 0)
+    p.lse[(static_cast<size_t>(b) * p.Hq + hq) * p.Nq + row] =
+        (l_tot > 0.f) ? (m_tot + log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
 }
 
 // One warp waits on an mbarrier nothing arrives on; the bounded wait runs out.
@@ -1107,8 +1095,6 @@ struct Plan {
   long long ws_bytes = 0;
 };
 
-constexpr long long kCtrBytes = 256;  // alignment of the partials after the counters
-
 static Plan make_plan(int B, int Hq, int Nq, int Nk, int causal, int d, int num_sms) {
   Plan pl;
   pl.n_qblk = (Nq + kRowsPerCta - 1) / kRowsPerCta;
@@ -1124,8 +1110,7 @@ static Plan make_plan(int B, int Hq, int Nq, int Nk, int causal, int d, int num_
   // a CTA's range holds at most two pieces of split units (its first and its
   // last), so two partial buffers per CTA cover every split
   const long long piece_bytes = 4LL * kTiles * kBlockM * (d + 2);
-  const long long ctr = ((4LL * pl.G + kCtrBytes - 1) / kCtrBytes) * kCtrBytes;
-  pl.ws_bytes = (pl.G > 1) ? ctr + 2LL * pl.G * piece_bytes : 0;
+  pl.ws_bytes = (pl.G > 1) ? 2LL * pl.G * piece_bytes : 0;
   return pl;
 }
 
@@ -1144,18 +1129,22 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
   static std::once_flag once;
   static int setup_status = FA2_OK;
   std::call_once(once, [] {
-    cudaFuncAttributes attr;
-    if (cudaFuncGetAttributes(&attr, fa2_fwd_kernel<D>) != cudaSuccess) {
-      setup_status = FA2_ERR_LAUNCH;
-      return;
+    for (auto* kern : {fa2_fwd_kernel<D, false>, fa2_fwd_kernel<D, true>}) {
+      cudaFuncAttributes attr;
+      if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) {
+        setup_status = FA2_ERR_LAUNCH;
+        return;
+      }
+      if (attr.numRegs != kLaunchRegs) {  // the setmaxnreg split assumes exactly this pool
+        setup_status = FA2_ERR_BUILD;
+        return;
+      }
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+          cudaSuccess) {
+        setup_status = FA2_ERR_LAUNCH;
+        return;
+      }
     }
-    if (attr.numRegs != kLaunchRegs) {  // the setmaxnreg split assumes exactly this pool
-      setup_status = FA2_ERR_BUILD;
-      return;
-    }
-    if (cudaFuncSetAttribute(fa2_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
-      setup_status = FA2_ERR_LAUNCH;
   });
   if (setup_status != FA2_OK) return setup_status;
 
@@ -1169,6 +1158,8 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
   p.Nk = Nk;
   p.causal = causal ? 1 : 0;
   p.n_qblk = (Nq + kRowsPerCta - 1) / kRowsPerCta;
+  p.r_empty = 0;
+  while (p.r_empty < p.n_qblk && unit_tiles(Nq, Nk, p.causal, p.n_qblk - 1 - p.r_empty) > 0) ++p.r_empty;
   // c is kept strictly positive so a masked score (-inf) always maps to
   // exp2(-inf) = 0; for softmax_scale == 0 every unmasked exponent is then
   // c * (s - m) ~ 1e-30 * O(1e4), which rounds to exp2(0) = 1 as required.
@@ -1181,7 +1172,6 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
   p.rem = 0;
   p.G = 1;
   p.ws = nullptr;
-  p.ws_ctr = nullptr;
   unsigned grid = static_cast<unsigned>(p.n_qblk) * Hq * B;  // one unit per CTA
   if (workspace) {
     const Plan pl = make_plan(B, Hq, Nq, Nk, p.causal, D, sm_count());
@@ -1193,9 +1183,7 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
       p.G = pl.G;
       p.span = static_cast<int>(pl.T / pl.G);
       p.rem = static_cast<int>(pl.T % pl.G);
-      p.ws_ctr = static_cast<int*>(workspace);
-      const long long ctr = ((4LL * pl.G + kCtrBytes - 1) / kCtrBytes) * kCtrBytes;
-      p.ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + ctr);
+      p.ws = static_cast<float*>(workspace);
       grid = static_cast<unsigned>(pl.G);
     }
   }
@@ -1204,8 +1192,17 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
   if (!encode_bnhd(&tq, q, B, Nq, Hq, D) || !encode_bnhd(&tk, k, B, Nk, Hkv, D) ||
       !encode_bnhd(&tv, v, B, Nk, Hkv, D))
     return FA2_ERR_LAUNCH;
-  fa2_fwd_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_LAUNCH;
+  if (p.streamk)
+    fa2_fwd_kernel<D, true><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  else
+    fa2_fwd_kernel<D, false><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return FA2_ERR_LAUNCH;
+  if (p.streamk && p.G > 1) {
+    const dim3 cgrid(static_cast<unsigned>(p.G - 1), kRowsPerCta / kCombineRows, D / 16);
+    fa2_combine_kernel<D><<<cgrid, kCombineThreads, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return FA2_ERR_LAUNCH;
+  }
+  return FA2_OK;
 }
 
 static int check_device() {

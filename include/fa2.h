@@ -85,35 +85,35 @@ int fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse
  * (the occupancy problem of "FlashAttention 2: Three Places the Chip Was Still
  * Waiting", section 2.3, and "FlashAttention-2 and -3: From Algebra to GPU
  * Scheduling", "Why more parallelism has limits").  fa2_forward_ws instead
- * launches one persistent block per SM and cuts the concatenated iterations of
- * all units (heaviest first) into equal contiguous ranges, one per block.  A
- * unit cut by a range boundary is computed in pieces over disjoint K/V
- * ranges; each piece keeps its own row max m and denominator l, and the last
- * piece to finish merges them with the identity that makes the softmax
- * statistics mergeable (m = max m_i, l = sum l_i e^(m_i - m),
- * O = sum O_i e^(m_i - m) / l): the same page, "Keep the unchanged
- * mathematical target in view" and "Another use of mergeable statistics".
- * Partials are kept in fp32, so the result equals fa2_forward's up to the
- * order of floating-point rounding.
+ * launches one persistent block per SM and cuts the summed unit costs (one
+ * per K/V tile plus a fixed per-unit cost for the pipeline fill and the
+ * epilogue; units heaviest first) into equal contiguous ranges, one per block.
+ * A unit cut by a range boundary is computed in pieces over disjoint K/V
+ * ranges; each piece writes its partial (O unnormalised in fp32, its row max
+ * m and denominator l) to the workspace, and a second kernel, launched by the
+ * same call on the same stream, merges the pieces of every split unit with
+ * the identity that makes the softmax statistics mergeable (m = max m_i,
+ * l = sum l_i e^(m_i - m), O = sum O_i e^(m_i - m) / l): the same page, "Keep
+ * the unchanged mathematical target in view" and "Another use of mergeable
+ * statistics".  This is the split-KV form of the forward pass; it also gives
+ * a single long unit (a short query block against a long key sequence) the
+ * whole GPU.  Partials stay in fp32 and are summed in a fixed order, so the
+ * result is deterministic and equals fa2_forward's up to the order of
+ * floating-point rounding.
  *
  *   workspace        device pointer, 16-byte aligned, at least
  *                    fa2_workspace_size(...) bytes for this problem on the
- *                    current device.  Its first fa2_workspace_size counters
- *                    (4 bytes per SM, rounded up to 256 bytes) must be zero
- *                    before the first call; every completed call leaves them
- *                    zero again, so one zero-fill at allocation suffices.
- *                    The rest is scratch the call overwrites.
+ *                    current device; scratch (no initialisation needed),
+ *                    overwritten by every call
  *   workspace_bytes  size of `workspace` in bytes
  *   (other arguments as in fa2_forward)
  *
  * Returns FA2_ERR_NULL_POINTER for a NULL workspace, FA2_ERR_WORKSPACE
  * when workspace_bytes is smaller than required, and FA2_ERR_SIZE when the
- * problem has 2^31 or more K/V-tile iterations in total (far beyond any
- * single call worth scheduling this way; fa2_forward has no such limit).  Calls that may run at the
- * same time (different streams without ordering between them) need separate
- * workspaces; calls ordered on one stream may share one.  A call that gave up
- * on a wait (see fa2_debug_status) may leave counters nonzero: zero the
- * workspace again before reusing it.
+ * summed unit costs reach 2^31 (far beyond any single call worth scheduling
+ * this way; fa2_forward has no such limit).  Calls that may run at the same
+ * time (streams without ordering between them) need separate workspaces;
+ * calls ordered on one stream may share one.
  */
 int fa2_forward_ws(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                    int Hkv, int Nq, int Nk, int d, int causal, float softmax_scale,
@@ -121,8 +121,8 @@ int fa2_forward_ws(const void* q, const void* k, const void* v, void* o, float* 
 
 /*
  * fa2_workspace_size -- bytes of workspace fa2_forward_ws needs for this
- * problem on the current device (0 when no unit is split, e.g. one SM's worth
- * of work).  Returns -1 for an invalid shape (as fa2_forward validates it),
+ * problem on the current device: two partials of 2 x 128 x (d + 2) floats per
+ * SM (0 when the work fits one block).  Returns -1 for an invalid shape (as fa2_forward validates it),
  * for a problem fa2_forward_ws refuses with FA2_ERR_SIZE, or when the device
  * cannot be queried.  Queries the device's SM count; makes no
  * other CUDA call.
@@ -153,7 +153,6 @@ enum fa2_wait_site {
   FA2_SITE_FINAL_STATS = 9,
   FA2_SITE_MMA_DRAIN = 10,
   FA2_SITE_LOAD_DRAIN = 11,
-  FA2_SITE_MERGE = 12,        /* stream-K: partial published / merge job hand-off */
   FA2_SITE_SELFTEST = 15
 };
 

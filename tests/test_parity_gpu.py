@@ -36,14 +36,11 @@ def sched(request):
     return request.param
 
 
-def counter_bytes(G):
-    return -(-4 * G // 256) * 256
-
-
 def run_gpu(fa2, q, k, v, causal, scale, guard=0, sched="units"):
     """Run the C-ABI forward on copies of q, k, v; O and LSE are carved out of
     NaN-filled buffers with `guard` poisoned elements on both sides.  Under
-    stream-K the workspace's counters must be back at zero afterwards."""
+    stream-K the workspace starts filled with NaN: it is scratch and must not
+    leak into the result."""
     dev = torch.device("cuda")
     qd, kd, vd = (t.to(dev).contiguous() for t in (q, k, v))
     B, Nq, Hq, d = q.shape
@@ -60,17 +57,12 @@ def run_gpu(fa2, q, k, v, causal, scale, guard=0, sched="units"):
                              torch.cuda.current_stream())
     else:
         ws = fa2.alloc_workspace(B, Hq, Hkv, Nq, Nk, d, causal, dev)
+        ws.fill_(0xFF)  # every float in it reads as NaN
         st = fa2.fa2_forward_ws(qd, kd, vd, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, ws,
                                 ws.numel(), torch.cuda.current_stream())
     assert st == 0, fa2.fa2_status_string(st)
     torch.cuda.synchronize()
     assert fa2.fa2_debug_status(None) == 0
-    if ws is not None:
-        sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        _, _, G, wsb = fa2.fa2_streamk_plan(B, Hq, Hkv, Nq, Nk, d, causal, sms)
-        assert wsb <= ws.numel()
-        if wsb:
-            assert int(ws[:counter_bytes(G)].count_nonzero()) == 0, "counters not reset"
     if guard:
         assert torch.isnan(o_buf[:g_o].float()).all() and torch.isnan(o_buf[-g_o:].float()).all(), \
             "O guard band overwritten"
@@ -227,14 +219,14 @@ def test_streamk_matches_units_closely(fa2):
 
 
 def test_workspace_reused_across_calls_and_shapes(fa2):
-    # one zero-filled workspace, sized for the largest problem, serves calls of
-    # different shapes ordered on one stream
+    # one workspace, sized for the largest problem, serves calls of different
+    # shapes ordered on one stream
     dev = torch.device("cuda")
     shapes = [Workload("r1", 2, 16, 16, 4096, 4096, 128, True, seed=24),
               Workload("r2", 1, 4, 2, 1000, 3000, 64, False, seed=25),
               Workload("r3", 2, 16, 16, 4096, 4096, 128, True, seed=24)]
     need = max(fa2.fa2_workspace_size(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal) for w in shapes)
-    ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=dev)
     outs = []
     for w in shapes:
         q, k, v = (t.to(dev) for t in make_qkv(w))
@@ -257,7 +249,7 @@ def test_small_workspace_is_refused(fa2):
     q, k, v = (t.to(dev) for t in make_qkv(w))
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
-    ws = torch.zeros(need - 256, dtype=torch.uint8, device=dev)
+    ws = torch.empty(need - 256, dtype=torch.uint8, device=dev)
     st = fa2.fa2_forward_ws(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
                             w.softmax_scale, ws, ws.numel(), torch.cuda.current_stream())
     assert st == 10

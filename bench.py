@@ -52,7 +52,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--schedule", default="streamk", choices=["streamk", "units"],
+    ap.add_argument("--schedule", default="units", choices=["units", "streamk"],
                     help="streamk: fa2_forward_ws, one persistent block per SM over a workspace; "
                          "units: fa2_forward, one block per (query block, head, batch)")
     return ap.parse_args()
@@ -247,7 +247,7 @@ def throughput_tflops(w, world: int, ms_per_step: float) -> float:
     return world * w.flops() / (ms_per_step * 1e-3) / 1e12
 
 
-def workload_config(w, n_gpus, schedule="streamk"):
+def workload_config(w, n_gpus, schedule="units"):
     return {"workload": w.name, "schedule": schedule, "description": w.description, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
             "Nq": w.Nq, "Nk": w.Nk, "d": w.d, "causal": w.causal,
             "softmax_scale": w.softmax_scale, "seed": w.seed,
@@ -279,10 +279,17 @@ def run_fa2(args, w):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    # stream-K needs a zero-filled workspace once; calls ordered on one stream reuse it
+    # stream-K takes a scratch workspace, allocated once; calls ordered on one
+    # stream reuse it.  It launches the persistent kernel and, when some unit
+    # is split, the combine kernel.
     ws = None
+    launches_per_step = 1
     if args.schedule == "streamk":
         ws = fa2.alloc_workspace(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal, dev)
+        _, _, ctas, _ = fa2.fa2_streamk_plan(
+            w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
+            torch.cuda.get_device_properties(dev).multi_processor_count)
+        launches_per_step = 2 if ctas > 1 else 1
 
     def call(qq, kk, vv, oo, ll):
         if ws is None:
@@ -395,10 +402,11 @@ def run_fa2(args, w):
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"bf16_tflops (burst, kernel timed alone), {peak_src}",
                          "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"]),
-                         "kernel": "fa2_fwd_kernel<128>" if w.d == 128 else "fa2_fwd_kernel<64>"},
+                         "kernel": f"fa2_fwd_kernel<{w.d}, {'true' if ws is not None else 'false'}>"
+                                   + (" + fa2_combine_kernel (timed together)" if launches_per_step > 1 else "")},
             "hbm_gbs_compulsory": w.compulsory_bytes() / (mean_ms * 1e-3) / 1e9,
             "bracket_ms_per_step_incl_flush": bracket_ms / args.steps,
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * launches_per_step,
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,

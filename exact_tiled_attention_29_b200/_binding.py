@@ -26,6 +26,7 @@ SITE_NAMES = {
     15: "SELFTEST",
 }
 FA2_SITE_SELFTEST = 15
+FA2_STATIC_WS_BYTES = 40 << 20  # the library's fixed stream-K scratch per device (fa2.h)
 
 
 class FA2Error(RuntimeError):
@@ -44,6 +45,8 @@ def _load() -> ctypes.CDLL:
     lib.fa2_forward.restype = ci
     lib.fa2_forward_ws.argtypes = [vp, vp, vp, vp, vp] + [ci] * 7 + [cf, vp, cll, vp]
     lib.fa2_forward_ws.restype = ci
+    lib.fa2_forward_static_ws.argtypes = [vp, vp, vp, vp, vp] + [ci] * 7 + [cf, vp]
+    lib.fa2_forward_static_ws.restype = ci
     lib.fa2_workspace_size.argtypes = [ci] * 7
     lib.fa2_workspace_size.restype = cll
     lib.fa2_status_string.argtypes = [ci]
@@ -98,6 +101,15 @@ def fa2_forward_ws(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale
                                    int(Hkv), int(Nq), int(Nk), int(d), int(bool(causal)),
                                    float(softmax_scale), _ptr(workspace), int(workspace_bytes),
                                    _stream(stream)))
+
+
+def fa2_forward_static_ws(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale,
+                          stream) -> int:
+    """Stream-K with the library's fixed scratch array; calls must not overlap."""
+    return int(_lib.fa2_forward_static_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B),
+                                          int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
+                                          int(bool(causal)), float(softmax_scale),
+                                          _stream(stream)))
 
 
 def fa2_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal) -> int:

@@ -1263,6 +1263,52 @@ extern "C" int fa2_forward_ws(const void* q, const void* k, const void* v, void*
                       workspace_bytes, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free stream-K: the same two kernels as fa2_forward_ws, with the
+// scratch taken from a fixed device array of this library instead of from
+// the caller.  For callers that cannot allocate device memory on the call
+// path and hold no buffer to lend: code running against a fixed, already
+// reserved memory budget (a serving loop that must not grow its footprint
+// per request), and code that cannot afford the device-wide synchronisation
+// cudaMalloc / cudaFree may imply.  Nothing in the array needs to start at
+// zero: every partial the combine kernel reads was written earlier in the
+// same call.  One array per device serves every call, so calls that may
+// overlap in time race on it.
+// ---------------------------------------------------------------------------
+constexpr size_t kStaticScratchBytes = FA2_STATIC_WS_BYTES;  // 2 partials x 148 SMs at d = 128 fit
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+// Device address of the array on device `dev` (the current device), looked
+// up once per device and cached; nullptr if the lookup failed.
+static void* static_scratch(int dev) {
+  static void* addr[64];
+  static std::once_flag flags[64];
+  std::call_once(flags[dev], [dev] {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_static_scratch) == cudaSuccess) addr[dev] = a;
+  });
+  return addr[dev];
+}
+
+extern "C" int fa2_forward_static_ws(const void* q, const void* k, const void* v, void* o, float* lse,
+                                     int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                                     float softmax_scale, void* stream) {
+  // the checks fa2_forward makes before touching CUDA, then the device
+  if (!q || !k || !v || !o || !lse) return FA2_ERR_NULL_POINTER;
+  const int sv = validate_shape(B, Hq, Hkv, Nq, Nk, d);
+  if (sv != FA2_OK) return sv;
+  if (!std::isfinite(softmax_scale)) return FA2_ERR_SCALE;
+  const int dv = check_device();
+  if (dv != FA2_OK) return dv;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FA2_ERR_DEVICE;
+  void* scratch = static_scratch(dev);
+  if (!scratch) return FA2_ERR_LAUNCH;
+  // a problem whose plan needs more than the array is refused (FA2_ERR_WORKSPACE)
+  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, scratch,
+                      static_cast<long long>(kStaticScratchBytes), stream);
+}
+
 extern "C" long long fa2_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal) {
   if (validate_shape(B, Hq, Hkv, Nq, Nk, d) != FA2_OK) return -1;
   const int n = sm_count();

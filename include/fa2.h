@@ -25,7 +25,8 @@
  *   - LSE is the natural log and includes softmax_scale.
  *
  * All entry points are thread-safe and allocate no device memory; the
- * stream-K variant takes its scratch memory from the caller.
+ * stream-K variant takes its scratch memory from the caller, or from a fixed
+ * array of the library (fa2_forward_static_ws, whose calls must not overlap).
  */
 #ifndef FA2_H
 #define FA2_H
@@ -128,6 +129,38 @@ int fa2_forward_ws(const void* q, const void* k, const void* v, void* o, float* 
  * other CUDA call.
  */
 long long fa2_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal);
+
+/*
+ * fa2_forward_static_ws -- fa2_forward_ws without a caller workspace: the
+ * stream-K scratch is a fixed device array inside this library
+ * (FA2_STATIC_WS_BYTES, 40 MiB per device, reserved when the library's device
+ * code is loaded on that device), so the call allocates no device memory and
+ * takes none from the caller.  The pages describe no such entry point; it has
+ * no counterpart there.  It is for callers that cannot allocate on the call
+ * path and hold no buffer to lend: code running inside a fixed, already
+ * reserved memory budget, or code that cannot afford the device-wide
+ * synchronisation that cudaMalloc / cudaFree may imply.
+ *
+ *   arguments, layouts and ownership as in fa2_forward.
+ *
+ * Nothing in the array needs to start at zero: every partial the merge reads
+ * is written earlier in the same call.  Returns FA2_ERR_WORKSPACE when the
+ * problem's fa2_workspace_size exceeds FA2_STATIC_WS_BYTES (it fits for
+ * d = 64 and d = 128 on GPUs with up to 157 SMs), FA2_ERR_LAUNCH when the
+ * array's device address cannot be obtained, and otherwise what
+ * fa2_forward_ws returns.
+ *
+ * The array's address is looked up once per device (cudaGetSymbolAddress,
+ * with that device current) on the first call on that device; make that first
+ * call before capturing the stream into a CUDA graph.  All calls on a device
+ * share the one array: calls that may overlap in time (unordered streams,
+ * several host threads) race on it and give wrong results -- order them on
+ * one stream.
+ */
+int fa2_forward_static_ws(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                          int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                          float softmax_scale, void* stream);
+#define FA2_STATIC_WS_BYTES (40LL << 20)
 
 /* Human-readable text for a status code (static storage, never NULL). */
 const char* fa2_status_string(int status);

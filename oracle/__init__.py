@@ -43,7 +43,7 @@ class Oracle:
         lib = ctypes.CDLL(so_path)
         f = lib.oracle_attention
         f.restype = ctypes.c_int
-        f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 7 + [ctypes.c_double] + \
+        f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 9 + [ctypes.c_double] + \
                      [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int] + \
                      [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
         lib.oracle_default_threads.restype = ctypes.c_int
@@ -53,11 +53,13 @@ class Oracle:
         return int(self._lib.oracle_default_threads())
 
     def attention(self, q, k, v, causal: bool, scale: float, rows=None, k_range=None,
-                  nthreads: int = 0):
+                  nthreads: int = 0, window=(-1, -1)):
         """Exact attention in fp64.
 
         q: uint16 [B,Nq,Hq,d] (bf16 bit patterns); k, v: uint16 [B,Nk,Hkv,d].
         rows: optional int sequence of query rows; k_range: optional (k_begin, k_end).
+        window: (left, right) widths of a local window around each row's
+        diagonal key i + Nk - Nq; a negative width leaves that side open.
         Returns (o [B,R,Hq,d] float64, lse [B,Hq,R] float64).
         """
         q = np.ascontiguousarray(q, dtype=np.uint16)
@@ -77,7 +79,8 @@ class Oracle:
         o = np.empty((B, n_rows, Hq, d), dtype=np.float64)
         lse = np.empty((B, Hq, n_rows), dtype=np.float64)
         rc = self._lib.oracle_attention(q.ctypes.data, k.ctypes.data, v.ctypes.data,
-                                        B, Hq, Hkv, Nq, Nk, d, int(bool(causal)), float(scale),
+                                        B, Hq, Hkv, Nq, Nk, d, int(bool(causal)),
+                                        int(window[0]), int(window[1]), float(scale),
                                         rows_ptr, n_rows, kb, ke,
                                         o.ctypes.data, lse.ctypes.data, int(nthreads))
         if rc != 0:
@@ -95,9 +98,11 @@ def _get() -> Oracle:
     return _default
 
 
-def attention(q, k, v, causal: bool, scale: float, rows=None, k_range=None, nthreads: int = 0):
+def attention(q, k, v, causal: bool, scale: float, rows=None, k_range=None, nthreads: int = 0,
+              window=(-1, -1)):
     """Module-level convenience over the default oracle build; see ``Oracle.attention``."""
-    return _get().attention(q, k, v, causal, scale, rows=rows, k_range=k_range, nthreads=nthreads)
+    return _get().attention(q, k, v, causal, scale, rows=rows, k_range=k_range, nthreads=nthreads,
+                            window=window)
 
 
 def default_threads() -> int:

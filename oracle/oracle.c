@@ -14,7 +14,10 @@
  *
  *   for every batch b, query head hq and query row i
  *     hk   = hq / (Hq / Hkv)                       (consecutive GQA groups)
- *     J_i  = { j in [k_begin, k_end) : not causal or j <= i + Nk - Nq }
+ *     g_i  = i + Nk - Nq                           (the row's diagonal key)
+ *     J_i  = { j in [k_begin, k_end) : not causal or j <= g_i,
+ *                                      wl < 0 or j >= g_i - wl,
+ *                                      wr < 0 or j <= g_i + wr }
  *     s_j  = scale * sum_c q[b,i,hq,c] * k[b,j,hk,c]     for j in J_i
  *     m    = max_j s_j
  *     w_j  = exp(s_j - m),   l = sum_j w_j
@@ -23,7 +26,10 @@
  *
  * The full score row is materialised (standard attention, the thing the
  * tiled method avoids); there is no tiling, no running max, no rescaling.
- * A row with an empty J_i gets O = 0 and LSE = -inf.
+ * A row with an empty J_i gets O = 0 and LSE = -inf.  wl / wr are the left /
+ * right widths of a sliding (local) window around the diagonal key, the
+ * sliding-window variant that forks from the same scheduling skeleton
+ * ("FlashAttention-2" explainer, "The Downstream Story"); -1 means no bound.
  *
  * Inputs are bf16 bit patterns; they are widened to double exactly.
  * Layouts: q [B,Nq,Hq,d], k and v [B,Nk,Hkv,d] (d contiguous).
@@ -40,6 +46,7 @@
 typedef struct {
     const uint16_t *q, *k, *v;
     int B, Hq, Hkv, Nq, Nk, d, causal;
+    int window_left, window_right; /* < 0: unbounded on that side */
     double scale;
     const int *rows;
     int n_rows;
@@ -64,6 +71,12 @@ static int key_visible(const oracle_job *J, int i, int j)
     if (j < J->k_begin || j >= J->k_end)
         return 0;
     if (J->causal && (long)j > (long)i + (long)J->Nk - (long)J->Nq)
+        return 0;
+    /* local window around the diagonal key g = i + Nk - Nq: g - wl <= j <= g + wr */
+    const long g = (long)J->Nk - (long)J->Nq + (long)i;
+    if (J->window_left >= 0 && (long)j < g - (long)J->window_left)
+        return 0;
+    if (J->window_right >= 0 && (long)j > g + (long)J->window_right)
         return 0;
     return 1;
 }
@@ -153,12 +166,15 @@ static void *oracle_worker(void *arg)
  * oracle_attention -- compute O and LSE for the rows listed in `rows`
  * (n_rows entries, indices into [0, Nq)), or for every row when rows == NULL
  * (then n_rows must equal Nq).  Keys are restricted to [k_begin, k_end)
- * intersected with the causal set; pass 0, Nk for the full range.
+ * intersected with the causal set and the window [g - window_left,
+ * g + window_right] around the diagonal key g = i + Nk - Nq (a negative width
+ * leaves that side open); pass 0, Nk and -1, -1 for the full range.
  * nthreads <= 0 uses every online core.  Returns 0 on success, 1 on bad
  * arguments, 2 on allocation or thread failure.
  */
 int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                     int window_left, int window_right,
                      double scale, const int *rows, int n_rows, int k_begin, int k_end,
                      double *o, double *lse, int nthreads)
 {
@@ -178,6 +194,8 @@ int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     oracle_job J;
     J.q = q; J.k = k; J.v = v;
     J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.Nq = Nq; J.Nk = Nk; J.d = d; J.causal = causal;
+    J.window_left = window_left < 0 ? -1 : window_left;
+    J.window_right = window_right < 0 ? -1 : window_right;
     J.scale = scale;
     J.rows = rows; J.n_rows = n_rows;
     J.k_begin = k_begin; J.k_end = k_end;

@@ -22,6 +22,17 @@ What pins what:
     math.exp / math.fsum on tiny inputs.
   * ``pin_invariants``   -- O is affine in V, the non-causal result is
     invariant to permuting the keys, and GQA equals explicitly repeated heads.
+  * ``pin_window_diagonal`` -- a local window of width (0, 0) leaves each row
+    exactly its diagonal key j = i + Nk - Nq: O equals that V row exactly and
+    LSE equals the one scaled score (rows whose diagonal lies outside the keys
+    get O = 0, LSE = -inf).
+  * ``pin_window_limits`` -- windows wider than both sequences reduce to the
+    pinned full cases: (wide, wide) is non-causal and (wide, 0) is causal,
+    bit for bit.
+  * ``pin_window_bruteforce`` -- the pure-Python evaluation with window
+    visibility, over left/right widths, causal and Nq != Nk.
+  * ``pin_window_merge`` -- a windowed result is the merge of its two key
+    halves (the mergeable-statistics identity again, under a window).
 """
 
 from __future__ import annotations
@@ -63,11 +74,21 @@ def _make(shape, seed, zero_q=False):
     return q, k, v
 
 
-def _visible(i, Nq, Nk, causal):
-    """Key indices the pages' causal rule leaves visible to row i (bottom-right aligned)."""
-    if not causal:
-        return list(range(Nk))
-    return [j for j in range(Nk) if j <= i + Nk - Nq]
+def _visible(i, Nq, Nk, causal, window=(-1, -1)):
+    """Key indices visible to row i: the causal rule (bottom-right aligned) and
+    a local window [g - left, g + right] around g = i + Nk - Nq, a negative
+    width leaving that side open."""
+    g = i + Nk - Nq
+    out = []
+    for j in range(Nk):
+        if causal and j > g:
+            continue
+        if window[0] >= 0 and j < g - window[0]:
+            continue
+        if window[1] >= 0 and j > g + window[1]:
+            continue
+        out.append(j)
+    return out
 
 
 def _f64(t):
@@ -254,5 +275,87 @@ def pin_invariants(orc):
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2), "GQA != repeated heads"
 
 
+def pin_window_diagonal(orc):
+    for shape in [(1, 2, 1, 9, 9, 8, False), (2, 2, 2, 5, 11, 4, True), (1, 2, 2, 12, 7, 8, False)]:
+        B, Hq, Hkv, Nq, Nk, d, causal = shape
+        q, k, v = _make(shape, 1000)
+        scale = 0.6
+        o, lse = _run(orc, q, k, v, causal, scale, window=(0, 0))
+        qd, kd, vd = _f64(q), _f64(k), _f64(v)
+        r = Hq // Hkv
+        for b in range(B):
+            for hq in range(Hq):
+                for i in range(Nq):
+                    g = i + Nk - Nq
+                    if not 0 <= g < Nk:
+                        assert np.all(o[b, i, hq] == 0) and lse[b, hq, i] == -np.inf
+                        continue
+                    assert np.array_equal(o[b, i, hq], vd[b, g, hq // r]), "window (0,0): O != V[g]"
+                    _close(lse[b, hq, i], scale * float(qd[b, i, hq] @ kd[b, g, hq // r]),
+                           what="window (0,0) LSE")
+
+
+def pin_window_limits(orc):
+    for shape in SHAPES:
+        B, Hq, Hkv, Nq, Nk, d, causal = shape
+        q, k, v = _make(shape, 1100)
+        wide = Nq + Nk
+        o_full, l_full = _run(orc, q, k, v, False, 0.5)
+        o_w, l_w = _run(orc, q, k, v, False, 0.5, window=(wide, wide))
+        assert np.array_equal(o_full, o_w) and np.array_equal(l_full, l_w), "wide window != full"
+        o_c, l_c = _run(orc, q, k, v, True, 0.5)
+        o_w, l_w = _run(orc, q, k, v, False, 0.5, window=(wide, 0))
+        assert np.array_equal(o_c, o_w) and np.array_equal(l_c, l_w), "(wide, 0) window != causal"
+
+
+def pin_window_bruteforce(orc):
+    cases = [((1, 2, 1, 9, 9, 4, True), (2, -1)), ((1, 2, 2, 7, 10, 3, False), (1, 2)),
+             ((2, 2, 1, 10, 6, 4, True), (3, -1)), ((1, 1, 1, 8, 8, 2, False), (-1, 1)),
+             ((1, 2, 2, 6, 9, 4, True), (0, -1))]
+    for shape, window in cases:
+        B, Hq, Hkv, Nq, Nk, d, causal = shape
+        q, k, v = _make(shape, 1200)
+        scale = 0.7
+        o, lse = _run(orc, q, k, v, causal, scale, window=window)
+        qq, kk, vv = q.float().tolist(), k.float().tolist(), v.float().tolist()
+        r = Hq // Hkv
+        for b in range(B):
+            for hq in range(Hq):
+                for i in range(Nq):
+                    vis = _visible(i, Nq, Nk, causal, window)
+                    if not vis:
+                        assert np.all(o[b, i, hq] == 0) and lse[b, hq, i] == -np.inf
+                        continue
+                    sc = [scale * math.fsum(qq[b][i][hq][c] * kk[b][j][hq // r][c] for c in range(d))
+                          for j in vis]
+                    big = max(sc)
+                    w = [math.exp(x - big) for x in sc]
+                    tot = math.fsum(w)
+                    ref = [math.fsum(w[t] * vv[b][j][hq // r][c] for t, j in enumerate(vis)) / tot
+                           for c in range(d)]
+                    _close(o[b, i, hq], ref, what=f"window {window} brute-force O")
+                    _close(lse[b, hq, i], big + math.log(tot), what=f"window {window} brute-force LSE")
+
+
+def pin_window_merge(orc):
+    shape = (2, 4, 2, 12, 16, 8, True)
+    B, Hq, Hkv, Nq, Nk, d, causal = shape
+    q, k, v = _make(shape, 1300)
+    for window in [(3, -1), (5, 2), (-1, 0)]:
+        o, lse = _run(orc, q, k, v, causal, 0.45, window=window)
+        oa, la = _run(orc, q, k, v, causal, 0.45, k_range=(0, 8), window=window)
+        ob, lb = _run(orc, q, k, v, causal, 0.45, k_range=(8, Nk), window=window)
+        m = np.maximum(la, lb)
+        safe = np.where(np.isfinite(m), m, 0.0)
+        tot = np.exp(la - safe) + np.exp(lb - safe)
+        l_ref = np.where(np.isfinite(m), safe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+        _close(lse, l_ref, what=f"window {window} merged LSE")
+        wa = np.where(np.isfinite(la), np.exp(la - np.where(np.isfinite(l_ref), l_ref, 0.0)), 0.0)
+        wb = np.where(np.isfinite(lb), np.exp(lb - np.where(np.isfinite(l_ref), l_ref, 0.0)), 0.0)
+        o_ref = (np.transpose(wa, (0, 2, 1))[..., None] * oa + np.transpose(wb, (0, 2, 1))[..., None] * ob)
+        _close(o, o_ref, tol=1e-11, what=f"window {window} merged O")
+
+
 ALL_PINS = [pin_zero_query, pin_single_key, pin_dominant_key, pin_merge, pin_library,
-            pin_bruteforce, pin_invariants]
+            pin_bruteforce, pin_invariants, pin_window_diagonal, pin_window_limits,
+            pin_window_bruteforce, pin_window_merge]

@@ -23,6 +23,9 @@ MUTANTS = [
     ("max_not_subtracted_in_weights", "s[j] = exp(s[j] - m);", "s[j] = exp(s[j] - m * 0.5);"),
     ("ignore_key_range", "if (j < J->k_begin || j >= J->k_end)", "if (0)"),
     ("q_row_index", "(((size_t)b * J->Nq + i) * J->Hq + hq) * d;", "(((size_t)b * J->Nq + ri) * J->Hq + hq) * d;"),
+    ("window_left_off_by_one", "(long)j < g - (long)J->window_left", "(long)j <= g - (long)J->window_left"),
+    ("window_right_ignored", "if (J->window_right >= 0 && (long)j > g + (long)J->window_right)", "if (0)"),
+    ("window_from_row_index", "const long g = (long)J->Nk - (long)J->Nq + (long)i;", "const long g = (long)i;"),
     ("drop_one_key_term", "for (int c = 0; c < d; ++c)\n            dot += qd[c]", "for (int c = 1; c < d; ++c)\n            dot += qd[c]"),
 ]
 

@@ -34,7 +34,10 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from exact_tiled_attention_29_b200.inputs import WORKLOADS, bf16_bits, make_qkv  # noqa: E402
+from exact_tiled_attention_29_b200.inputs import (EXTRA_WORKLOADS, WORKLOADS, bf16_bits,  # noqa: E402
+                                                  make_qkv)
+
+ALL_WORKLOADS = {**WORKLOADS, **EXTRA_WORKLOADS}
 
 METRIC = "attention fwd TFLOP/s (bf16, 1 B200) and % of dense BF16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -47,7 +50,7 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="causal_8k", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="causal_8k", choices=sorted(ALL_WORKLOADS))
     ap.add_argument("--impl", default="fa2", choices=["fa2", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -164,16 +167,29 @@ def oracle_sample_rows(w, seconds: float, orc, q, k, v):
     # calibrate on a handful of rows spread over the sequence
     cal = np.linspace(0, w.Nq - 1, 16).astype(np.int32)
     t0 = time.perf_counter()
-    orc.attention(q, k, v, w.causal, w.softmax_scale, rows=cal)
+    orc.attention(q, k, v, w.causal, w.softmax_scale, rows=cal, window=window_of(w))
     dt = max(time.perf_counter() - t0, 1e-4)
     per_row = dt / (len(cal) * w.B * w.Hq)
     n = int(max(8, min(w.Nq, seconds / per_row / (w.B * w.Hq))))
     return np.unique(np.linspace(0, w.Nq - 1, n).astype(np.int32))
 
 
+def window_of(w):
+    return (w.window_left, w.window_right)
+
+
 def sample_flops(w, rows) -> float:
-    vis = [(min(int(r) + w.Nk - w.Nq, w.Nk - 1) + 1) if w.causal else w.Nk for r in rows]
-    vis = [max(0, x) for x in vis]
+    """Algorithmic FLOPs of the sampled rows: 4 d per visible (row, key) pair."""
+    vis = []
+    for r in rows:
+        g = int(r) + w.Nk - w.Nq
+        hi = w.Nk - 1
+        if w.causal:
+            hi = min(hi, g)
+        if w.window_right >= 0:
+            hi = min(hi, g + w.window_right)
+        lo = max(0, g - w.window_left) if w.window_left >= 0 else 0
+        vis.append(max(0, hi - lo + 1))
     return 4.0 * w.d * w.B * w.Hq * float(sum(vis))
 
 
@@ -183,7 +199,7 @@ def cpu_oracle_baseline(w, seconds: float):
     q, k, v = (bf16_bits(t) for t in make_qkv(w))
     rows = oracle_sample_rows(w, seconds, orc, q, k, v)
     t0 = time.perf_counter()
-    orc.attention(q, k, v, w.causal, w.softmax_scale, rows=rows)
+    orc.attention(q, k, v, w.causal, w.softmax_scale, rows=rows, window=window_of(w))
     dt = time.perf_counter() - t0
     fl = sample_flops(w, rows)
     return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": orc.default_threads(),
@@ -204,10 +220,10 @@ def run_reference(args, w):
     rows = oracle_sample_rows(w, per_step, orc, q, k, v)
     fl = sample_flops(w, rows)
     for _ in range(args.warmup):
-        orc.attention(q, k, v, w.causal, w.softmax_scale, rows=rows)
+        orc.attention(q, k, v, w.causal, w.softmax_scale, rows=rows, window=window_of(w))
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        orc.attention(q, k, v, w.causal, w.softmax_scale, rows=rows)
+        orc.attention(q, k, v, w.causal, w.softmax_scale, rows=rows, window=window_of(w))
     dt = (time.perf_counter() - t0) / max(1, args.steps)
     val = fl / dt / 1e12
     sample = (f"{len(rows)} evenly spaced query rows x all {w.B * w.Hq} (batch, head) pairs of "
@@ -248,8 +264,11 @@ def throughput_tflops(w, world: int, ms_per_step: float) -> float:
 
 
 def workload_config(w, n_gpus, schedule="units"):
-    return {"workload": w.name, "schedule": schedule, "description": w.description, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
-            "Nq": w.Nq, "Nk": w.Nk, "d": w.d, "causal": w.causal,
+    cfg = {"workload": w.name, "schedule": schedule, "description": w.description, "B": w.B,
+           "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nk": w.Nk, "d": w.d, "causal": w.causal}
+    if w.windowed:
+        cfg["window"] = [w.window_left, w.window_right]
+    return {**cfg,
             "softmax_scale": w.softmax_scale, "seed": w.seed,
             "flops_per_step_per_rank": w.flops(),
             "parallelism": f"independent batches per rank x{n_gpus}" if n_gpus > 1 else "single GPU",
@@ -284,6 +303,8 @@ def run_fa2(args, w):
     # is split, the combine kernel.
     ws = None
     launches_per_step = 1
+    if args.schedule == "streamk" and w.windowed:
+        raise SystemExit("the local-window workloads run the one-block-per-unit schedule only")
     if args.schedule == "streamk":
         ws = fa2.alloc_workspace(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal, dev)
         _, _, ctas, _ = fa2.fa2_streamk_plan(
@@ -292,7 +313,11 @@ def run_fa2(args, w):
         launches_per_step = 2 if ctas > 1 else 1
 
     def call(qq, kk, vv, oo, ll):
-        if ws is None:
+        if w.windowed:
+            st = fa2.fa2_forward_local(qq, kk, vv, oo, ll, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d,
+                                       w.window_left, 0 if w.causal else w.window_right,
+                                       w.softmax_scale, stream)
+        elif ws is None:
             st = fa2.fa2_forward(qq, kk, vv, oo, ll, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
                                  w.softmax_scale, stream)
         else:
@@ -422,7 +447,7 @@ def run_fa2(args, w):
 
 def main():
     args = parse_args()
-    w = WORKLOADS[args.workload]
+    w = ALL_WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
     return run_fa2(args, w)

@@ -18,7 +18,7 @@ FA2_OK = 0
 STATUS_NAMES = {
     0: "FA2_OK", 1: "FA2_ERR_NULL_POINTER", 2: "FA2_ERR_BAD_SHAPE", 3: "FA2_ERR_HEAD_DIM",
     4: "FA2_ERR_ALIGNMENT", 5: "FA2_ERR_SCALE", 6: "FA2_ERR_DEVICE", 7: "FA2_ERR_LAUNCH",
-    8: "FA2_ERR_SIZE", 9: "FA2_ERR_BUILD", 10: "FA2_ERR_WORKSPACE",
+    8: "FA2_ERR_SIZE", 9: "FA2_ERR_BUILD", 10: "FA2_ERR_WORKSPACE", 11: "FA2_ERR_WINDOW",
 }
 SITE_NAMES = {
     1: "Q_LOADED", 2: "KV_LOADED", 3: "KV_FREE", 4: "S_READY", 5: "P_READY", 6: "STATS_READY",
@@ -45,6 +45,8 @@ def _load() -> ctypes.CDLL:
     lib.fa2_forward.restype = ci
     lib.fa2_forward_ws.argtypes = [vp, vp, vp, vp, vp] + [ci] * 7 + [cf, vp, cll, vp]
     lib.fa2_forward_ws.restype = ci
+    lib.fa2_forward_local.argtypes = [vp, vp, vp, vp, vp] + [ci] * 8 + [cf, vp]
+    lib.fa2_forward_local.restype = ci
     lib.fa2_forward_static_ws.argtypes = [vp, vp, vp, vp, vp] + [ci] * 7 + [cf, vp]
     lib.fa2_forward_static_ws.restype = ci
     lib.fa2_workspace_size.argtypes = [ci] * 7
@@ -92,6 +94,15 @@ def fa2_forward(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, s
     return int(_lib.fa2_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(Hq),
                                 int(Hkv), int(Nq), int(Nk), int(d), int(bool(causal)),
                                 float(softmax_scale), _stream(stream)))
+
+
+def fa2_forward_local(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, window_left, window_right,
+                      softmax_scale, stream) -> int:
+    """Local (sliding-window) attention; -1 leaves a side open.  Returns the status code."""
+    return int(_lib.fa2_forward_local(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B),
+                                      int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
+                                      int(window_left), int(window_right), float(softmax_scale),
+                                      _stream(stream)))
 
 
 def fa2_forward_ws(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, workspace,
@@ -164,13 +175,14 @@ def alloc_workspace(B, Hq, Hkv, Nq, Nk, d, causal, device):
 
 
 def attention(q, k, v, causal: bool = False, softmax_scale: float | None = None, out=None,
-              lse=None, stream=None, workspace=None):
+              lse=None, stream=None, workspace=None, window=None):
     """O, LSE for bf16 CUDA tensors q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d] (contiguous).
 
     Outputs are allocated with torch unless given; the work is one call to
     ``fa2_forward`` on ``stream`` (default: torch's current stream), or to
     ``fa2_forward_ws`` (stream-K schedule) when ``workspace`` -- a CUDA tensor
-    from ``alloc_workspace`` -- is given.
+    from ``alloc_workspace`` -- is given, or to ``fa2_forward_local`` when
+    ``window`` = (left, right) is given (causal then narrows the right side to 0).
     """
     import torch
 
@@ -189,7 +201,16 @@ def attention(q, k, v, causal: bool = False, softmax_scale: float | None = None,
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    if workspace is None:
+    if window is not None:
+        if workspace is not None:
+            raise ValueError("the local-window path has no stream-K variant")
+        wl, wr = int(window[0]), int(window[1])
+        if causal:  # j <= g and j <= g + wr (wr >= 0) is j <= g
+            wr = 0
+        st = fa2_forward_local(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, wl, wr, softmax_scale,
+                               stream)
+        where = "fa2_forward_local"
+    elif workspace is None:
         st = fa2_forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, stream)
         where = "fa2_forward"
     else:

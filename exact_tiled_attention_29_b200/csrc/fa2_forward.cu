@@ -115,7 +115,7 @@ struct Params {
   __nv_bfloat16* o;
   float* lse;
   int B, Hq, Hkv, Nq, Nk;
-  int causal;
+  int wl, wr;         // visibility window widths (see Window); causal is (-1, 0)
   int n_qblk;
   int r_empty;        // first round (heaviest first) of units with no visible key; n_qblk if none
   float c;            // |softmax_scale| * log2(e)
@@ -130,25 +130,60 @@ struct Params {
   float* ws;          // stream-K partials: [G CTAs][2: first / last piece of its range][piece floats]
 };
 
-// Number of K/V tiles a 128-row query tile starting at row r0 visits (0 if it
-// has no valid row or no visible key).
-__host__ __device__ inline int kv_tiles_for(int Nq, int Nk, int causal, int r0) {
+// Visibility: key j is visible to query row i when g - wl <= j <= g + wr
+// with g = i + Nk - Nq, the row's diagonal key (bottom-right alignment); a
+// negative width leaves that side open.  Causal attention is (-1, 0), full
+// attention (-1, -1), and a sliding (local) window ("FlashAttention-2"
+// explainer, "The Downstream Story") bounds the left side too.
+struct Window {
+  int wl, wr;
+};
+
+// K/V tiles a 128-row query tile starting at row r0 can see: [lo, lo + count)
+// (count 0 when no row of it sees any key).
+// (32-bit arithmetic: the host keeps 2 (Nq + Nk) below 2^31 and clamps the
+// widths below Nk / Nq.)
+__host__ __device__ inline int tile_span(int Nq, int Nk, Window w, int r0, int& lo) {
+  lo = 0;
   if (r0 >= Nq) return 0;
-  const int nkt = (Nk + kBlockN - 1) / kBlockN;
-  if (!causal) return nkt;
-  const int rlast = (r0 + kBlockM - 1 < Nq - 1) ? r0 + kBlockM - 1 : Nq - 1;
-  const long long lim = (long long)rlast + (long long)Nk - (long long)Nq;  // last visible key of the last row
-  if (lim < 0) return 0;
-  const long long t = lim / kBlockN + 1;
-  return t < nkt ? (int)t : nkt;
+  const int koff = Nk - Nq;
+  const int rl = (r0 + kBlockM - 1 < Nq - 1) ? r0 + kBlockM - 1 : Nq - 1;
+  int first = (w.wl >= 0) ? r0 + koff - w.wl : 0;      // left bound of the first row
+  int last = (w.wr >= 0) ? rl + koff + w.wr : Nk - 1;  // right bound of the last row
+  if (first < 0) first = 0;
+  if (last > Nk - 1) last = Nk - 1;
+  if (first > last) return 0;
+  lo = first / kBlockN;
+  return last / kBlockN - lo + 1;
 }
 
-// K/V tiles of a unit (query block qb): the longer of its two query tiles.
-__host__ __device__ inline int unit_tiles(int Nq, int Nk, int causal, int qb) {
-  const int a = kv_tiles_for(Nq, Nk, causal, qb * kRowsPerCta);
-  const int b = kv_tiles_for(Nq, Nk, causal, qb * kRowsPerCta + kBlockM);
-  return a > b ? a : b;
+// A unit's K/V range: it starts at tile j0, the first tile either of its two
+// query tiles sees, and query tile t needs its first n0 / n1 tiles.  A query
+// tile whose window starts later meets fully masked tiles first; they cost an
+// iteration and contribute nothing.
+struct UnitSpan {
+  int j0, n0, n1;
+};
+__host__ __device__ inline UnitSpan unit_span(int Nq, int Nk, Window w, int qb) {
+  int lo0 = 0, lo1 = 0;
+  const int c0 = tile_span(Nq, Nk, w, qb * kRowsPerCta, lo0);
+  const int c1 = tile_span(Nq, Nk, w, qb * kRowsPerCta + kBlockM, lo1);
+  UnitSpan u{0, 0, 0};
+  if (c0 == 0 && c1 == 0) return u;
+  u.j0 = (c0 > 0 && c1 > 0) ? (lo0 < lo1 ? lo0 : lo1) : (c0 > 0 ? lo0 : lo1);
+  u.n0 = c0 > 0 ? lo0 + c0 - u.j0 : 0;
+  u.n1 = c1 > 0 ? lo1 + c1 - u.j0 : 0;
+  return u;
 }
+
+// K/V-tile iterations of a unit (query block qb).
+__host__ __device__ inline int unit_tiles(int Nq, int Nk, Window w, int qb) {
+  const UnitSpan u = unit_span(Nq, Nk, w, qb);
+  return u.n0 > u.n1 ? u.n0 : u.n1;
+}
+
+__host__ __device__ inline Window window_of(const Params& p) { return Window{p.wl, p.wr}; }
+inline Window causal_window(int causal) { return Window{-1, causal ? 0 : -1}; }
 
 // Start of CTA c's iteration range, floor(c * T / G), in 32-bit arithmetic:
 // c*T/G = c*span + c*rem/G with T = span*G + rem, c*span <= T < 2^31 and
@@ -172,6 +207,7 @@ __host__ __device__ inline int range_start(int span, int rem, int G, int c) {
 // ---------------------------------------------------------------------------
 struct Piece {
   int b, hq, qb;
+  int j0;           // first K/V tile of the unit (absolute); iterations count from it
   int jb, je;       // K/V tiles [jb, je) of the unit
   int nt0, nt1;     // K/V tiles of Q0 / Q1 over the whole unit
   int a0, a1;       // iterations of Q0 / Q1 in this piece
@@ -217,8 +253,10 @@ struct PieceIter {
     pc.hq = k % p.Hq;
     pc.jb = jb;
     pc.je = je;
-    pc.nt0 = kv_tiles_for(p.Nq, p.Nk, p.causal, pc.qb * kRowsPerCta);
-    pc.nt1 = kv_tiles_for(p.Nq, p.Nk, p.causal, pc.qb * kRowsPerCta + kBlockM);
+    const UnitSpan u = unit_span(p.Nq, p.Nk, window_of(p), pc.qb);
+    pc.j0 = u.j0;
+    pc.nt0 = u.n0;
+    pc.nt1 = u.n1;
     pc.a0 = max(0, min(je, pc.nt0) - jb);
     pc.a1 = max(0, min(je, pc.nt1) - jb);
   }
@@ -256,11 +294,11 @@ struct PieceIter {
   __device__ __forceinline__ void seek_round(const Params& p, int pos) {
     r = 0;
     cum = 0;
-    n = unit_tiles(p.Nq, p.Nk, p.causal, p.n_qblk - 1);
+    n = unit_tiles(p.Nq, p.Nk, window_of(p), p.n_qblk - 1);
     while (pos >= cum + HB * cost(n)) {  // the end of a round is at most T < 2^31
       cum += HB * cost(n);
       ++r;
-      n = unit_tiles(p.Nq, p.Nk, p.causal, p.n_qblk - 1 - r);
+      n = unit_tiles(p.Nq, p.Nk, window_of(p), p.n_qblk - 1 - r);
     }
   }
 
@@ -294,7 +332,7 @@ struct PieceIter {
       const int u = blockIdx.x;
       r = u / HB;
       k_cur = u % HB;
-      const int nn = unit_tiles(p.Nq, p.Nk, p.causal, p.n_qblk - 1 - r);
+      const int nn = unit_tiles(p.Nq, p.Nk, window_of(p), p.n_qblk - 1 - r);
       if (nn == 0) return false;  // nothing to compute: the merge warps write this unit's empty rows
       cum = 0;
       n = nn;
@@ -314,7 +352,7 @@ struct PieceIter {
       while (x >= cum + HB * cost(n)) {
         cum += HB * cost(n);
         ++r;
-        n = unit_tiles(p.Nq, p.Nk, p.causal, p.n_qblk - 1 - r);
+        n = unit_tiles(p.Nq, p.Nk, window_of(p), p.n_qblk - 1 - r);
       }
     }
     const int w = cost(n);
@@ -446,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m_sc = 0.f;         // m_raw * c (0 while no key was visible)
       float l = 0.f;            // running denominator, relative to m_sc
       for (int jj = 0; jj < ntt; ++jj) {
-        const int j = pc.jb + jj;  // K/V tile of the unit
+        const int j = pc.j0 + pc.jb + jj;  // K/V tile (absolute)
         if (!mbar_wait_warp(bar(BAR_S + t), s_cnt & 1, g, FA2_SITE_S_READY, j)) {
           ok = false;
           break;
@@ -462,16 +500,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i) s[32 * k + i] = __uint_as_float(r[i]);
         }
         tmem_wait_ld();
-        // causal diagonal / ragged key tail: only these tiles pay for masking
+        // window edges (the causal diagonal) and the ragged key tail: only
+        // tiles some row's bound falls into pay for masking
         const int kbase = j * kBlockN;
-        const bool masked = (kbase + kBlockN > p.Nk) || (p.causal && kbase + kBlockN - 1 > r0t + koff);
-        int lim = kBlockN - 1;  // last visible column of this tile for this row
+        const bool masked = (kbase + kBlockN > p.Nk) ||
+                            (p.wr >= 0 && kbase + kBlockN - 1 > r0t + koff + p.wr) ||
+                            (p.wl >= 0 && kbase < r0t + kBlockM - 1 + koff - p.wl);
         if (masked) {
-          lim = min(lim, p.Nk - 1 - kbase);
-          if (p.causal) lim = min(lim, row + koff - kbase);
+          // visible columns [lo, hi] of this tile for this row (64-bit: the
+          // window bounds may lie far outside the tile)
+          const long long gk = static_cast<long long>(row) + koff - kbase;  // diagonal key, tile-relative
+          long long hi = min(kBlockN - 1, p.Nk - 1 - kbase);
+          if (p.wr >= 0 && gk + p.wr < hi) hi = gk + p.wr;
+          const long long lo = (p.wl >= 0) ? gk - p.wl : 0;
+          const int hi_i = static_cast<int>(hi < -1 ? -1 : hi);
+          const int lo_i = static_cast<int>(lo > kBlockN ? kBlockN : lo);
 #pragma unroll
           for (int i = 0; i < kBlockN; ++i)
-            if (i > lim) s[i] = -INFINITY;
+            if (i > hi_i || i < lo_i) s[i] = -INFINITY;
         }
         // row max: 8 independent chains of 3-input max (max is exact in any order)
         float mp[8];
@@ -855,7 +901,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         ++pieces;
-        for (int j = pc.jb; j < pc.je && ok; ++j) {
+        for (int j = pc.j0 + pc.jb; j < pc.j0 + pc.je && ok; ++j) {  // absolute K/V tiles
 #pragma unroll 1
           for (int kv = 0; kv < 2; ++kv, ++it) {
             const int st = static_cast<int>(it % C::kStages);
@@ -1075,6 +1121,7 @@ static int validate_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
   const long long q_bytes = 2LL * B * Nq * Hq * d;
   const long long kv_bytes = 2LL * B * Nk * Hkv * d;
   if (q_bytes >= lim || kv_bytes >= lim) return FA2_ERR_SIZE;
+  if (static_cast<long long>(Nq) + Nk >= (1LL << 30)) return FA2_ERR_SIZE;  // window bounds stay in int
   const long long nblk = (static_cast<long long>(Nq) + kRowsPerCta - 1) / kRowsPerCta;
   if (nblk * Hq * B > INT_MAX) return FA2_ERR_SIZE;
   // one round of units (all heads and batches of a query block) must count
@@ -1095,13 +1142,13 @@ struct Plan {
   long long ws_bytes = 0;
 };
 
-static Plan make_plan(int B, int Hq, int Nq, int Nk, int causal, int d, int num_sms) {
+static Plan make_plan(int B, int Hq, int Nq, int Nk, Window win, int d, int num_sms) {
   Plan pl;
   pl.n_qblk = (Nq + kRowsPerCta - 1) / kRowsPerCta;
   const long long HB = static_cast<long long>(B) * Hq;
   pl.units = HB * pl.n_qblk;
   for (int qb = 0; qb < pl.n_qblk; ++qb) {
-    const int n = unit_tiles(Nq, Nk, causal, qb);
+    const int n = unit_tiles(Nq, Nk, win, qb);
     pl.iters += HB * n;
     pl.T += HB * (n > 0 ? n + kUnitCost : 0);
   }
@@ -1123,7 +1170,7 @@ static int sm_count() {
 
 template <int D>
 static int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                  int Hkv, int Nq, int Nk, int causal, float scale, void* workspace,
+                  int Hkv, int Nq, int Nk, Window win, float scale, void* workspace,
                   long long workspace_bytes, cudaStream_t stream) {
   using C = Cfg<D>;
   static std::once_flag once;
@@ -1156,10 +1203,11 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
   p.Hkv = Hkv;
   p.Nq = Nq;
   p.Nk = Nk;
-  p.causal = causal ? 1 : 0;
+  p.wl = win.wl;
+  p.wr = win.wr;
   p.n_qblk = (Nq + kRowsPerCta - 1) / kRowsPerCta;
   p.r_empty = 0;
-  while (p.r_empty < p.n_qblk && unit_tiles(Nq, Nk, p.causal, p.n_qblk - 1 - p.r_empty) > 0) ++p.r_empty;
+  while (p.r_empty < p.n_qblk && unit_tiles(Nq, Nk, win, p.n_qblk - 1 - p.r_empty) > 0) ++p.r_empty;
   // c is kept strictly positive so a masked score (-inf) always maps to
   // exp2(-inf) = 0; for softmax_scale == 0 every unmasked exponent is then
   // c * (s - m) ~ 1e-30 * O(1e4), which rounds to exp2(0) = 1 as required.
@@ -1174,7 +1222,7 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
   p.ws = nullptr;
   unsigned grid = static_cast<unsigned>(p.n_qblk) * Hq * B;  // one unit per CTA
   if (workspace) {
-    const Plan pl = make_plan(B, Hq, Nq, Nk, p.causal, D, sm_count());
+    const Plan pl = make_plan(B, Hq, Nq, Nk, win, D, sm_count());
     if (pl.G > 0) {  // otherwise every unit is empty: one CTA per unit writes it
       if (pl.T > INT_MAX) return FA2_ERR_SIZE;
       if (workspace_bytes < pl.ws_bytes) return FA2_ERR_WORKSPACE;
@@ -1225,7 +1273,7 @@ static int check_device() {
 using namespace fa2;
 
 static int forward_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                        int Hq, int Hkv, int Nq, int Nk, int d, int causal, float softmax_scale,
+                        int Hq, int Hkv, int Nq, int Nk, int d, Window win, float softmax_scale,
                         void* workspace, long long workspace_bytes, void* stream) {
   if (!q || !k || !v || !o || !lse) return FA2_ERR_NULL_POINTER;
   const int sv = validate_shape(B, Hq, Hkv, Nq, Nk, d);
@@ -1241,17 +1289,27 @@ static int forward_impl(const void* q, const void* k, const void* v, void* o, fl
   if (dv != FA2_OK) return dv;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 128)
-    return launch<128>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal, softmax_scale, workspace,
+    return launch<128>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, win, softmax_scale, workspace,
                        workspace_bytes, s);
-  return launch<64>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, causal, softmax_scale, workspace,
+  return launch<64>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, win, softmax_scale, workspace,
                     workspace_bytes, s);
 }
 
 extern "C" int fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                            int Hq, int Hkv, int Nq, int Nk, int d, int causal, float softmax_scale,
                            void* stream) {
-  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, nullptr, 0,
-                      stream);
+  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal_window(causal), softmax_scale,
+                      nullptr, 0, stream);
+}
+
+extern "C" int fa2_forward_local(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 int B, int Hq, int Hkv, int Nq, int Nk, int d, int window_left,
+                                 int window_right, float softmax_scale, void* stream) {
+  if (window_left < -1 || window_right < -1) return FA2_ERR_WINDOW;
+  // a width that reaches past every key of every row is no bound: g - wl <= 0
+  // for all rows once wl >= Nk, and g + wr >= Nk - 1 once wr >= Nq
+  Window w{window_left >= Nk ? -1 : window_left, window_right >= Nq ? -1 : window_right};
+  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, w, softmax_scale, nullptr, 0, stream);
 }
 
 extern "C" int fa2_forward_ws(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -1259,8 +1317,8 @@ extern "C" int fa2_forward_ws(const void* q, const void* k, const void* v, void*
                               float softmax_scale, void* workspace, long long workspace_bytes,
                               void* stream) {
   if (!workspace) return FA2_ERR_NULL_POINTER;
-  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, workspace,
-                      workspace_bytes, stream);
+  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal_window(causal), softmax_scale,
+                      workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -1305,15 +1363,15 @@ extern "C" int fa2_forward_static_ws(const void* q, const void* k, const void* v
   void* scratch = static_scratch(dev);
   if (!scratch) return FA2_ERR_LAUNCH;
   // a problem whose plan needs more than the array is refused (FA2_ERR_WORKSPACE)
-  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, scratch,
-                      static_cast<long long>(kStaticScratchBytes), stream);
+  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal_window(causal), softmax_scale,
+                      scratch, static_cast<long long>(kStaticScratchBytes), stream);
 }
 
 extern "C" long long fa2_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal) {
   if (validate_shape(B, Hq, Hkv, Nq, Nk, d) != FA2_OK) return -1;
   const int n = sm_count();
   if (n <= 0) return -1;
-  const Plan pl = make_plan(B, Hq, Nq, Nk, causal ? 1 : 0, d, n);
+  const Plan pl = make_plan(B, Hq, Nq, Nk, causal_window(causal), d, n);
   return pl.T > INT_MAX ? -1 : pl.ws_bytes;
 }
 
@@ -1323,7 +1381,7 @@ extern "C" int fa2_streamk_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, i
   const int sv = validate_shape(B, Hq, Hkv, Nq, Nk, d);
   if (sv != FA2_OK) return sv;
   if (num_sms <= 0) return FA2_ERR_BAD_SHAPE;
-  const Plan pl = make_plan(B, Hq, Nq, Nk, causal ? 1 : 0, d, num_sms);
+  const Plan pl = make_plan(B, Hq, Nq, Nk, causal_window(causal), d, num_sms);
   if (pl.T > INT_MAX) return FA2_ERR_SIZE;
   if (total_iters) *total_iters = pl.iters;
   if (ctas) *ctas = pl.G;
@@ -1344,6 +1402,7 @@ extern "C" const char* fa2_status_string(int status) {
     case FA2_ERR_SIZE: return "problem exceeds the supported tensor or grid extent";
     case FA2_ERR_BUILD: return "kernel image does not match its register plan";
     case FA2_ERR_WORKSPACE: return "workspace smaller than fa2_workspace_size reports";
+    case FA2_ERR_WINDOW: return "window widths must be >= -1";
     default: return "unknown status";
   }
 }

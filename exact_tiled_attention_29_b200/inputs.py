@@ -39,6 +39,14 @@ class Workload:
     outlier_frac: float = 0.0
     outlier_scale: float = 8.0
     description: str = field(default="", compare=False)
+    # local (sliding-window) attention: key j visible to row i iff
+    # g - window_left <= j <= g + window_right, g = i + Nk - Nq; -1 = open side
+    window_left: int = -1
+    window_right: int = -1
+
+    @property
+    def windowed(self) -> bool:
+        return self.window_left >= 0 or self.window_right >= 0
 
     @property
     def softmax_scale(self) -> float:
@@ -49,9 +57,25 @@ class Workload:
 
     # ---- bookkeeping used by the benchmark (counts, not attention math) ----
     def flops(self) -> float:
-        """Algorithmic FLOPs: 4*B*Hq*Nq*Nk*d, halved when causal."""
-        f = 4.0 * self.B * self.Hq * self.Nq * self.Nk * self.d
-        return f / 2.0 if self.causal else f
+        """Algorithmic FLOPs: 4*B*Hq*Nq*Nk*d, halved when causal; with a window,
+        4*B*Hq*d per visible (query, key) pair, counted exactly."""
+        if not self.windowed:
+            f = 4.0 * self.B * self.Hq * self.Nq * self.Nk * self.d
+            return f / 2.0 if self.causal else f
+        return 4.0 * self.B * self.Hq * self.d * float(self.visible_pairs())
+
+    def visible_pairs(self) -> int:
+        """Number of visible (query row, key) pairs of one head (a count of index ranges)."""
+        g = np.arange(self.Nq, dtype=np.int64) + (self.Nk - self.Nq)
+        hi = np.full(self.Nq, self.Nk - 1, dtype=np.int64)
+        lo = np.zeros(self.Nq, dtype=np.int64)
+        if self.causal:
+            hi = np.minimum(hi, g)
+        if self.window_right >= 0:
+            hi = np.minimum(hi, g + self.window_right)
+        if self.window_left >= 0:
+            lo = np.maximum(lo, g - self.window_left)
+        return int(np.maximum(hi - lo + 1, 0).sum())
 
     def compulsory_bytes(self) -> int:
         """Read Q, K, V once (bf16), write O once (bf16) and LSE (fp32)."""
@@ -76,6 +100,13 @@ WORKLOADS = {
                                      "1% of Q/K entries x8"),
     "gqa_4k": Workload("gqa_4k", 4, 32, 8, 4096, 4096, 128, True,
                        description="GQA causal, B=4 Hq=32 Hkv=8 N=4096 d=128"),
+}
+
+# Further workloads for the variants built on the same path (not among the
+# five above): local attention with a causal window of 1024 keys per row.
+EXTRA_WORKLOADS = {
+    "local_8k": Workload("local_8k", 2, 16, 16, 8192, 8192, 128, True, window_left=1023,
+                         description="causal sliding window of 1024 keys, B=2 H=16 N=8192 d=128"),
 }
 
 

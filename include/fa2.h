@@ -47,7 +47,8 @@ enum fa2_status_code {
   FA2_ERR_LAUNCH = 7,         /* a CUDA runtime/driver call or the launch failed    */
   FA2_ERR_SIZE = 8,           /* a tensor or the grid exceeds the supported extent   */
   FA2_ERR_BUILD = 9,          /* the kernel image does not match its register plan  */
-  FA2_ERR_WORKSPACE = 10      /* workspace smaller than fa2_workspace_size reports   */
+  FA2_ERR_WORKSPACE = 10,     /* workspace smaller than fa2_workspace_size reports   */
+  FA2_ERR_WINDOW = 11         /* a window width below -1                             */
 };
 
 /*
@@ -75,6 +76,27 @@ enum fa2_status_code {
  */
 int fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                 int Hkv, int Nq, int Nk, int d, int causal, float softmax_scale, void* stream);
+
+/*
+ * fa2_forward_local -- local (sliding-window) attention: as fa2_forward, with
+ * key j visible to query row i exactly when
+ *
+ *     g - window_left <= j <= g + window_right,   g = i + Nk - Nq
+ *
+ * (g is the row's diagonal key under the bottom-right alignment used for
+ * causal attention).  A width of -1 leaves that side open: (-1, 0) is causal
+ * attention, (-1, -1) full attention, (W, 0) a causal window of W + 1 keys.
+ * The sliding-window variants fork from the same scheduling skeleton
+ * ("FlashAttention-2" explainer, "The Downstream Story"); here the window
+ * narrows each query block's range of K/V tiles (tiles wholly outside every
+ * row's window are never loaded or multiplied) and only tiles that a row's
+ * bound falls into pay for masking.  Rows that see no key get O = 0 and
+ * LSE = -inf.  Returns FA2_ERR_WINDOW for a width below -1; otherwise as
+ * fa2_forward.
+ */
+int fa2_forward_local(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int Hq, int Hkv, int Nq, int Nk, int d, int window_left, int window_right,
+                      float softmax_scale, void* stream);
 
 /*
  * fa2_forward_ws -- the same computation as fa2_forward, scheduled stream-K

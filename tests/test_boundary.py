@@ -58,6 +58,14 @@ def test_validation_status_codes(over, code):
     assert fa2.fa2_status_string(code) not in ("", "unknown status")
 
 
+def test_local_window_validation():
+    args = (16, 32, 48, 64, 80, 1, 2, 1, 5, 7, 128)
+    assert fa2.fa2_forward_local(*args, -2, 0, 0.1, None) == 11
+    assert fa2.fa2_forward_local(*args, 0, -5, 0.1, None) == 11
+    assert fa2.fa2_forward_local(0, 32, 48, 64, 80, 1, 2, 1, 5, 7, 128, 3, 0, 0.1, None) == 1
+    assert fa2.fa2_forward_local(16, 32, 48, 64, 80, 1, 2, 1, 5, 7, 80, 3, 0, 0.1, None) == 3
+
+
 def test_valid_arguments_reach_the_device_check_only():
     import torch
     st = call()
@@ -67,7 +75,7 @@ def test_valid_arguments_reach_the_device_check_only():
 
 
 def test_status_strings():
-    for code in range(11):
+    for code in range(12):
         assert isinstance(fa2.fa2_status_string(code), str)
     assert fa2.fa2_status_string(12345) == "unknown status"
 

@@ -103,8 +103,12 @@ WORKLOADS = {
 }
 
 # Further workloads for the variants built on the same path (not among the
-# five above): local attention with a causal window of 1024 keys per row.
+# five above): local attention with a causal window of 1024 keys per row, and
+# a short query block against a long key sequence (16 units of 256 K/V tiles:
+# one block per unit leaves most SMs idle; the split-KV schedule does not).
 EXTRA_WORKLOADS = {
+    "shortq_32k": Workload("shortq_32k", 1, 16, 16, 256, 32768, 128, False,
+                           description="short query vs long keys, B=1 H=16 Nq=256 Nk=32768 d=128"),
     "local_8k": Workload("local_8k", 2, 16, 16, 8192, 8192, 128, True, window_left=1023,
                          description="causal sliding window of 1024 keys, B=2 H=16 N=8192 d=128"),
 }

@@ -47,6 +47,10 @@ class Oracle:
                      [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int] + \
                      [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
         lib.oracle_default_threads.restype = ctypes.c_int
+        b = lib.oracle_attention_backward
+        b.restype = ctypes.c_int
+        b.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9 + [ctypes.c_double] + \
+                     [ctypes.c_void_p] * 3 + [ctypes.c_int]
         self._lib = lib
 
     def default_threads(self) -> int:
@@ -88,6 +92,30 @@ class Oracle:
         return o, lse
 
 
+    def backward(self, q, k, v, dout, causal: bool, scale: float, window=(-1, -1),
+                 nthreads: int = 0):
+        """Gradients of the attention output against an upstream gradient, in fp64.
+
+        q, dout: uint16 [B,Nq,Hq,d] (bf16 bit patterns); k, v: uint16 [B,Nk,Hkv,d].
+        Returns (dq [B,Nq,Hq,d], dk [B,Nk,Hkv,d], dv [B,Nk,Hkv,d]) float64.
+        """
+        q, k, v, dout = (np.ascontiguousarray(t, dtype=np.uint16) for t in (q, k, v, dout))
+        B, Nq, Hq, d = q.shape
+        Bk, Nk, Hkv, dk_ = k.shape
+        if v.shape != k.shape or dout.shape != q.shape or Bk != B or dk_ != d:
+            raise ValueError("shape mismatch between q, k, v, dout")
+        dq = np.empty((B, Nq, Hq, d), dtype=np.float64)
+        dk = np.empty((B, Nk, Hkv, d), dtype=np.float64)
+        dv = np.empty((B, Nk, Hkv, d), dtype=np.float64)
+        rc = self._lib.oracle_attention_backward(
+            q.ctypes.data, k.ctypes.data, v.ctypes.data, dout.ctypes.data, B, Hq, Hkv, Nq, Nk, d,
+            int(bool(causal)), int(window[0]), int(window[1]), float(scale), dq.ctypes.data,
+            dk.ctypes.data, dv.ctypes.data, int(nthreads))
+        if rc != 0:
+            raise ValueError(f"oracle_attention_backward rejected its arguments (status {rc})")
+        return dq, dk, dv
+
+
 _default: Oracle | None = None
 
 
@@ -103,6 +131,11 @@ def attention(q, k, v, causal: bool, scale: float, rows=None, k_range=None, nthr
     """Module-level convenience over the default oracle build; see ``Oracle.attention``."""
     return _get().attention(q, k, v, causal, scale, rows=rows, k_range=k_range, nthreads=nthreads,
                             window=window)
+
+
+def backward(q, k, v, dout, causal: bool, scale: float, window=(-1, -1), nthreads: int = 0):
+    """Module-level convenience over the default oracle build; see ``Oracle.backward``."""
+    return _get().backward(q, k, v, dout, causal, scale, window=window, nthreads=nthreads)
 
 
 def default_threads() -> int:

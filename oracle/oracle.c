@@ -238,3 +238,164 @@ int oracle_default_threads(void)
     long n = sysconf(_SC_NPROCESSORS_ONLN);
     return n < 1 ? 1 : (n > 256 ? 256 : (int)n);
 }
+
+/* ------------------------------------------------------------------------
+ * Backward pass (gradients of the attention output), from the definition.
+ *
+ * With P_ij = exp(s_ij - m_i) / l_i the probabilities of row i over its
+ * visible keys J_i, O_i = sum_j P_ij v_j and an upstream gradient dO:
+ *
+ *   dV_j  = sum_i P_ij dO_i                         (over the rows i that see j)
+ *   dP_ij = dO_i . v_j
+ *   dS_ij = P_ij (dP_ij - sum_k P_ik dP_ik)         (the softmax Jacobian)
+ *   dQ_i  = scale * sum_j dS_ij k_j
+ *   dK_j  = scale * sum_i dS_ij q_i
+ *
+ * summed over the query heads of a KV head's group for dK and dV.  The
+ * pages' headline numbers are forward+backward training numbers and name the
+ * backward pass as the forward's counterpart ("FlashAttention 2: Three Places
+ * the Chip Was Still Waiting", section 2.5); its arithmetic here is the chain
+ * rule applied to the plain definition above, with no tiling and no
+ * recomputation tricks.  dq is [B,Nq,Hq,d], dk and dv are [B,Nk,Hkv,d], all
+ * double.  Returns 0, 1 on bad arguments, 2 on allocation or thread failure.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    const oracle_job *J;
+    const uint16_t *dout;
+    double *dq, *dk, *dv;
+    long next_group;  /* (b, hk) work counter, advanced atomically */
+} oracle_bwd_job;
+
+/* All query heads of one (batch, KV head) group: every row's probabilities,
+ * then its dQ row and its contributions to the group's dK and dV rows. */
+static void backward_group(const oracle_bwd_job *W, int b, int hk, double *p, double *dp)
+{
+    const oracle_job *J = W->J;
+    const int d = J->d, group = J->Hq / J->Hkv;
+    for (int hq = hk * group; hq < (hk + 1) * group; ++hq) {
+        for (int i = 0; i < J->Nq; ++i) {
+            const size_t row_at = (((size_t)b * J->Nq + i) * J->Hq + hq) * (size_t)d;
+            const uint16_t *qrow = J->q + row_at;
+            const uint16_t *gorow = W->dout + row_at;
+            double *dqrow = W->dq + row_at;
+            for (int c = 0; c < d; ++c)
+                dqrow[c] = 0.0;
+            double m = -INFINITY;
+            int n_visible = 0;
+            for (int j = 0; j < J->Nk; ++j) {
+                if (!key_visible(J, i, j))
+                    continue;
+                const uint16_t *krow = J->k + (((size_t)b * J->Nk + j) * J->Hkv + hk) * d;
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c)
+                    dot += bf16_to_double(qrow[c]) * bf16_to_double(krow[c]);
+                p[j] = J->scale * dot;
+                if (p[j] > m)
+                    m = p[j];
+                ++n_visible;
+            }
+            if (n_visible == 0)
+                continue;
+            double l = 0.0;
+            for (int j = 0; j < J->Nk; ++j) {
+                if (!key_visible(J, i, j))
+                    continue;
+                p[j] = exp(p[j] - m);
+                l += p[j];
+            }
+            double pdp = 0.0; /* sum_k P_ik dP_ik */
+            for (int j = 0; j < J->Nk; ++j) {
+                if (!key_visible(J, i, j))
+                    continue;
+                p[j] /= l;
+                const uint16_t *vj = J->v + (((size_t)b * J->Nk + j) * J->Hkv + hk) * d;
+                double g = 0.0;
+                for (int c = 0; c < d; ++c)
+                    g += bf16_to_double(gorow[c]) * bf16_to_double(vj[c]);
+                dp[j] = g;
+                pdp += p[j] * g;
+            }
+            for (int j = 0; j < J->Nk; ++j) {
+                if (!key_visible(J, i, j))
+                    continue;
+                const double ds = p[j] * (dp[j] - pdp);
+                const uint16_t *krow = J->k + (((size_t)b * J->Nk + j) * J->Hkv + hk) * d;
+                double *dkrow = W->dk + (((size_t)b * J->Nk + j) * J->Hkv + hk) * d;
+                double *dvrow = W->dv + (((size_t)b * J->Nk + j) * J->Hkv + hk) * d;
+                for (int c = 0; c < d; ++c) {
+                    dqrow[c] += J->scale * ds * bf16_to_double(krow[c]);
+                    dkrow[c] += J->scale * ds * bf16_to_double(qrow[c]);
+                    dvrow[c] += p[j] * bf16_to_double(gorow[c]);
+                }
+            }
+        }
+    }
+}
+
+static void *oracle_bwd_worker(void *arg)
+{
+    oracle_bwd_job *W = (oracle_bwd_job *)arg;
+    const oracle_job *J = W->J;
+    double *p = (double *)malloc(sizeof(double) * (size_t)J->Nk);
+    double *dp = (double *)malloc(sizeof(double) * (size_t)J->Nk);
+    if (!p || !dp) {
+        free(p);
+        free(dp);
+        return (void *)1;
+    }
+    const long n_groups = (long)J->B * J->Hkv;
+    for (;;) {
+        long it = __atomic_fetch_add(&W->next_group, 1, __ATOMIC_RELAXED);
+        if (it >= n_groups)
+            break;
+        backward_group(W, (int)(it / J->Hkv), (int)(it % J->Hkv), p, dp);
+    }
+    free(p);
+    free(dp);
+    return NULL;
+}
+
+int oracle_attention_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                              const uint16_t *dout, int B, int Hq, int Hkv, int Nq, int Nk,
+                              int d, int causal, int window_left, int window_right, double scale,
+                              double *dq, double *dk, double *dv, int nthreads)
+{
+    if (!q || !k || !v || !dout || !dq || !dk || !dv)
+        return 1;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0 || d > 512 || Hq % Hkv != 0)
+        return 1;
+    oracle_job J;
+    memset(&J, 0, sizeof J);
+    J.q = q; J.k = k; J.v = v;
+    J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.Nq = Nq; J.Nk = Nk; J.d = d; J.causal = causal;
+    J.window_left = window_left < 0 ? -1 : window_left;
+    J.window_right = window_right < 0 ? -1 : window_right;
+    J.scale = scale;
+    J.k_begin = 0; J.k_end = Nk;
+    memset(dk, 0, sizeof(double) * (size_t)B * Nk * Hkv * d);
+    memset(dv, 0, sizeof(double) * (size_t)B * Nk * Hkv * d);
+    oracle_bwd_job W;
+    W.J = &J; W.dout = dout; W.dq = dq; W.dk = dk; W.dv = dv; W.next_group = 0;
+    int nt = nthreads > 0 ? nthreads : oracle_default_threads();
+    const long n_groups = (long)B * Hkv;
+    if (nt > n_groups)
+        nt = (int)n_groups;
+    pthread_t tid[256];
+    int started = 0, rc = 0;
+    for (int t = 1; t < nt && t < 256; ++t) {
+        if (pthread_create(&tid[started], NULL, oracle_bwd_worker, &W) != 0) {
+            rc = 2;
+            break;
+        }
+        ++started;
+    }
+    if (oracle_bwd_worker(&W) != NULL)
+        rc = 2;
+    for (int t = 0; t < started; ++t) {
+        void *ret = NULL;
+        pthread_join(tid[t], &ret);
+        if (ret != NULL)
+            rc = 2;
+    }
+    return rc;
+}

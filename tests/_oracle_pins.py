@@ -359,3 +359,123 @@ def pin_window_merge(orc):
 ALL_PINS = [pin_zero_query, pin_single_key, pin_dominant_key, pin_merge, pin_library,
             pin_bruteforce, pin_invariants, pin_window_diagonal, pin_window_limits,
             pin_window_bruteforce, pin_window_merge]
+
+
+# ---------------------------------------------------------------------------
+# Backward pass (gradients), pinned to calculus and to a library:
+#   * ``pin_bwd_finite_difference`` -- central differences of the scalar
+#     L = sum(G * O) of a plain fp64 forward (numpy, masked softmax) agree with
+#     the oracle's dQ, dK, dV at sampled elements.
+#   * ``pin_bwd_autograd`` -- torch autograd through scaled_dot_product_attention
+#     in fp64 (explicit mask, enable_gqa).
+#   * ``pin_bwd_single_key`` -- window (0, 0): every row sees one key, P = 1,
+#     so dS = 0 (dQ = dK = 0 exactly) and dV_j is the plain sum of the dO rows
+#     whose diagonal key is j.
+#   * ``pin_bwd_gqa`` -- GQA equals the repeated-head problem with dK, dV summed
+#     over each group.
+# ---------------------------------------------------------------------------
+
+def _run_bwd(orc, q, k, v, g, causal, scale, **kw):
+    return orc.backward(bf16_bits(q), bf16_bits(k), bf16_bits(v), bf16_bits(g), causal, scale, **kw)
+
+
+def _forward_np(q, k, v, causal, scale, window=(-1, -1)):
+    """Plain masked-softmax attention in fp64 numpy ([B,N,H,d] layouts)."""
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    r = Hq // Hkv
+    o = np.zeros_like(q)
+    for b in range(B):
+        for h in range(Hq):
+            s = scale * q[b, :, h] @ k[b, :, h // r].T
+            for i in range(Nq):
+                vis = _visible(i, Nq, Nk, causal, window)
+                mask = np.full(Nk, -np.inf)
+                mask[vis] = 0.0
+                row = s[i] + mask
+                if not vis:
+                    continue
+                w = np.exp(row - row.max())
+                o[b, i, h] = (w / w.sum()) @ v[b, :, h // r]
+    return o
+
+
+def pin_bwd_finite_difference(orc):
+    for shape, window in [((1, 2, 1, 7, 9, 4, True), (-1, -1)), ((1, 2, 2, 6, 6, 3, False), (2, 1))]:
+        B, Hq, Hkv, Nq, Nk, d, causal = shape
+        q, k, v = _make(shape, 2000)
+        g = _randn_bf16((B, Nq, Hq, d), torch.Generator().manual_seed(2001))
+        scale = 0.55
+        dq, dk, dv = _run_bwd(orc, q, k, v, g, causal, scale, window=window)
+        qd, kd, vd, gd = _f64(q), _f64(k), _f64(v), _f64(g)
+        loss = lambda qq, kk, vv: float((gd * _forward_np(qq, kk, vv, causal, scale, window)).sum())
+        eps = 1e-5
+        rng = np.random.default_rng(2002)
+        for name, base, grad in (("dQ", qd, dq), ("dK", kd, dk), ("dV", vd, dv)):
+            for _ in range(12):
+                idx = tuple(int(rng.integers(n)) for n in base.shape)
+                args_p = [qd.copy(), kd.copy(), vd.copy()]
+                args_m = [qd.copy(), kd.copy(), vd.copy()]
+                which = "QKV".index(name[1])
+                args_p[which][idx] += eps
+                args_m[which][idx] -= eps
+                fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+                assert abs(fd - grad[idx]) <= 1e-7 * max(1.0, abs(fd)), \
+                    f"{name}{idx}: finite difference {fd} vs oracle {grad[idx]}"
+
+
+def pin_bwd_autograd(orc):
+    for shape in [(2, 4, 2, 9, 17, 8, True), (1, 2, 2, 11, 11, 8, False), (1, 4, 1, 17, 9, 8, True)]:
+        B, Hq, Hkv, Nq, Nk, d, causal = shape
+        q, k, v = _make(shape, 2100)
+        g = _randn_bf16((B, Nq, Hq, d), torch.Generator().manual_seed(2101))
+        scale = 0.4
+        dq, dk, dv = _run_bwd(orc, q, k, v, g, causal, scale)
+        qt = q.double().permute(0, 2, 1, 3).requires_grad_(True)
+        kt = k.double().permute(0, 2, 1, 3).requires_grad_(True)
+        vt = v.double().permute(0, 2, 1, 3).requires_grad_(True)
+        mask = torch.ones(Nq, Nk, dtype=torch.bool)
+        if causal:
+            mask = torch.tensor([[j <= i + Nk - Nq for j in range(Nk)] for i in range(Nq)])
+        out = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale,
+                                                               enable_gqa=True)
+        # rows with no visible key: the oracle's convention (O = 0) has zero gradient
+        keep = mask.any(dim=1)
+        out = torch.where(keep[None, None, :, None], out, torch.zeros_like(out))
+        out.backward(g.double().permute(0, 2, 1, 3))
+        _close(dq, qt.grad.permute(0, 2, 1, 3).numpy(), tol=1e-11, what="autograd dQ")
+        _close(dk, kt.grad.permute(0, 2, 1, 3).numpy(), tol=1e-11, what="autograd dK")
+        _close(dv, vt.grad.permute(0, 2, 1, 3).numpy(), tol=1e-11, what="autograd dV")
+
+
+def pin_bwd_single_key(orc):
+    shape = (2, 4, 2, 9, 12, 8, False)
+    B, Hq, Hkv, Nq, Nk, d, causal = shape
+    q, k, v = _make(shape, 2200)
+    g = _randn_bf16((B, Nq, Hq, d), torch.Generator().manual_seed(2201))
+    dq, dk, dv = _run_bwd(orc, q, k, v, g, False, 0.9, window=(0, 0))
+    assert np.all(dq == 0) and np.all(dk == 0), "one visible key: dS must vanish"
+    gd = _f64(g)
+    ref = np.zeros_like(dv)
+    r = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(Nq):
+                ref[b, i + Nk - Nq, h // r] += gd[b, i, h]
+    _close(dv, ref, what="one visible key: dV = sum of dO rows")
+
+
+def pin_bwd_gqa(orc):
+    shape = (2, 6, 2, 9, 11, 8, True)
+    B, Hq, Hkv, Nq, Nk, d, causal = shape
+    q, k, v = _make(shape, 2300)
+    g = _randn_bf16((B, Nq, Hq, d), torch.Generator().manual_seed(2301))
+    dq1, dk1, dv1 = _run_bwd(orc, q, k, v, g, True, 0.5)
+    r = Hq // Hkv
+    dq2, dk2, dv2 = _run_bwd(orc, q, k.repeat_interleave(r, dim=2), v.repeat_interleave(r, dim=2), g, True, 0.5)
+    _close(dq1, dq2, tol=1e-13, what="GQA dQ")
+    _close(dk1, dk2.reshape(B, Nk, Hkv, r, d).sum(axis=3), tol=1e-13, what="GQA dK")
+    _close(dv1, dv2.reshape(B, Nk, Hkv, r, d).sum(axis=3), tol=1e-13, what="GQA dV")
+
+
+BWD_PINS = [pin_bwd_finite_difference, pin_bwd_autograd, pin_bwd_single_key, pin_bwd_gqa]

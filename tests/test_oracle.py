@@ -12,6 +12,11 @@ def test_oracle_pin(oracle_lib, pin):
     pin(oracle_lib)
 
 
+@pytest.mark.parametrize("pin", pins.BWD_PINS, ids=lambda p: p.__name__)
+def test_oracle_backward_pin(oracle_lib, pin):
+    pin(oracle_lib)
+
+
 def test_oracle_rejects_bad_arguments(oracle_lib):
     q = np.zeros((1, 4, 3, 8), np.uint16)
     k = np.zeros((1, 4, 2, 8), np.uint16)

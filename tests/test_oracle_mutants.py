@@ -30,6 +30,44 @@ MUTANTS = [
 ]
 
 
+# mistakes in the backward pass, caught by the backward pins
+BWD_MUTANTS = [
+    ("bwd_dq_without_scale", "dqrow[c] += J->scale * ds * bf16_to_double(krow[c]);",
+     "dqrow[c] += ds * bf16_to_double(krow[c]);"),
+    ("bwd_ds_without_row_term", "const double ds = p[j] * (dp[j] - pdp);", "const double ds = p[j] * dp[j];"),
+    ("bwd_dk_from_k", "dkrow[c] += J->scale * ds * bf16_to_double(qrow[c]);",
+     "dkrow[c] += J->scale * ds * bf16_to_double(krow[c]);"),
+    ("bwd_dv_unnormalised", "                p[j] /= l;\n", "                p[j] /= 1.0;\n"),
+    ("bwd_dv_uses_ds", "dvrow[c] += p[j] * bf16_to_double(gorow[c]);", "dvrow[c] += dp[j] * bf16_to_double(gorow[c]);"),
+    ("bwd_dp_from_q", "g += bf16_to_double(gorow[c]) * bf16_to_double(vj[c]);",
+     "g += bf16_to_double(gorow[c]) * bf16_to_double(qrow[c]);"),
+    ("bwd_one_head_per_group", "for (int hq = hk * group; hq < (hk + 1) * group; ++hq) {",
+     "for (int hq = hk * group; hq < hk * group + 1; ++hq) {"),
+]
+
+
+def _mutant_fails_some_pin(tmp_path, name, old, new, pin_list):
+    text = open(SRC).read()
+    assert text.count(old) == 1, f"mutation site for {name} not found exactly once"
+    src = tmp_path / "oracle_mut.c"
+    src.write_text(text.replace(old, new))
+    so = oracle.build(force=True, src=str(src), out=str(tmp_path / "liboracle_mut.so"))
+    orc = oracle.Oracle(so)
+    failed = []
+    for pin in pin_list:
+        try:
+            pin(orc)
+        except AssertionError:
+            failed.append(pin.__name__)
+    return failed
+
+
+@pytest.mark.parametrize("name,old,new", BWD_MUTANTS, ids=[m[0] for m in BWD_MUTANTS])
+def test_backward_pins_catch_mutant(tmp_path, name, old, new):
+    assert _mutant_fails_some_pin(tmp_path, name, old, new, pins.BWD_PINS), \
+        f"mutant {name} passed every backward pin"
+
+
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_pins_catch_mutant(tmp_path, name, old, new):
     text = open(SRC).read()

@@ -49,6 +49,10 @@ def _load() -> ctypes.CDLL:
     lib.fa2_forward_local.restype = ci
     lib.fa2_forward_static_ws.argtypes = [vp, vp, vp, vp, vp] + [ci] * 7 + [cf, vp]
     lib.fa2_forward_static_ws.restype = ci
+    lib.fa2_backward.argtypes = [vp] * 9 + [ci] * 7 + [cf, vp, cll, vp]
+    lib.fa2_backward.restype = ci
+    lib.fa2_backward_workspace_size.argtypes = [ci] * 4
+    lib.fa2_backward_workspace_size.restype = cll
     lib.fa2_workspace_size.argtypes = [ci] * 7
     lib.fa2_workspace_size.restype = cll
     lib.fa2_status_string.argtypes = [ci]
@@ -121,6 +125,19 @@ def fa2_forward_static_ws(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softma
                                           int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
                                           int(bool(causal)), float(softmax_scale),
                                           _stream(stream)))
+
+
+def fa2_backward(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale,
+                 workspace, workspace_bytes, stream) -> int:
+    """Gradients dq, dk, dv of the forward pass (fp32 scratch in `workspace`).  Returns the status."""
+    return int(_lib.fa2_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                                 _ptr(dk), _ptr(dv), int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
+                                 int(bool(causal)), float(softmax_scale), _ptr(workspace),
+                                 int(workspace_bytes), _stream(stream)))
+
+
+def fa2_backward_workspace_size(B, Hq, Nq, d) -> int:
+    return int(_lib.fa2_backward_workspace_size(int(B), int(Hq), int(Nq), int(d)))
 
 
 def fa2_workspace_size(B, Hq, Hkv, Nq, Nk, d, causal) -> int:
@@ -220,3 +237,28 @@ def attention(q, k, v, causal: bool = False, softmax_scale: float | None = None,
     if st != FA2_OK:
         raise FA2Error(st, where)
     return out, lse
+
+
+def attention_backward(q, k, v, o, lse, dout, causal: bool = False,
+                       softmax_scale: float | None = None, stream=None, workspace=None):
+    """dq, dk, dv for bf16 CUDA tensors (layouts as ``attention``) given the
+    forward's o and lse and the upstream gradient dout; one call to
+    ``fa2_backward``.  ``workspace`` (uint8 CUDA tensor of at least
+    ``fa2_backward_workspace_size`` bytes) is allocated with torch if absent."""
+    import torch
+
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    if workspace is None:
+        workspace = torch.empty(fa2_backward_workspace_size(B, Hq, Nq, d), dtype=torch.uint8,
+                                device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    st = fa2_backward(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal,
+                      softmax_scale, workspace, workspace.numel() * workspace.element_size(), stream)
+    if st != FA2_OK:
+        raise FA2Error(st, "fa2_backward")
+    return dq, dk, dv

@@ -1,0 +1,505 @@
+// fa2_backward.cuh -- backward pass of exact attention (dQ, dK, dV) for sm_100a.
+//
+// Included by fa2_forward.cu, inside namespace fa2: one translation unit, so
+// both passes share the bounded-wait status word and the helpers above.
+//
+// Given the forward's O and LSE and an upstream gradient dO, with
+// P_ij = exp(scale * q_i . k_j - LSE_i) over the keys row i sees:
+//
+//   D_i   = dO_i . O_i                     (= sum_j P_ij dP_ij)
+//   dV_j  = sum_i P_ij dO_i
+//   dP_ij = dO_i . v_j,   dS_ij = P_ij (dP_ij - D_i)
+//   dQ_i  = scale * sum_j dS_ij k_j,   dK_j = scale * sum_i dS_ij q_i
+//
+// ("FlashAttention 2: Three Places the Chip Was Still Waiting", section 2.5
+// reports the forward+backward figures; the gradients are the chain rule on
+// the forward's definition.)  As in the forward, nothing of size Nq x Nk is
+// stored: P is recomputed tile by tile from the saved LSE.
+//
+// Work decomposition: one CTA per (128-key block, KV head, batch) owns dK and
+// dV of its keys in tensor memory for the whole pass and walks every query
+// tile of every query head of its group that sees any of its keys, so dK and
+// dV need no atomics (GQA sums the group's heads in place).  dQ is the only
+// output shared between CTAs: each CTA adds its 128 x d contribution per
+// query tile into an fp32 accumulator with vector atomics, and a last kernel
+// scales nothing (scale is applied before the atomics) and rounds it to bf16.
+//
+// Per query tile (tensor memory: S^T | dP^T | dV | dK):
+//   MMA   S^T = K Q^T (SS), dP^T = V dO^T (SS)            -> "S ready"
+//   WG0   P^T = exp2(S^T c - LSE_i log2 e), dS^T = P^T (dP^T - D_i),
+//         both written back to tensor memory as bf16 over S^T / dP^T, and
+//         dS^T into shared memory as the MN-major A operand of dQ -> "P ready"
+//   MMA   dV += P^T dO (TS), dK += dS^T Q (TS), dQ_tile = dS K (SS, into the
+//         S^T columns, after the dV MMA read P^T: one thread's MMAs run in
+//         issue order)                                     -> "dQ ready"
+//   WG1   read dQ_tile, scale, add into the fp32 accumulator -> "dQ free"
+//   and the next tile's S^T may overwrite the columns.
+//
+// Roles: warps 0-3 (WG0) P / dS, one thread per key row; warps 4-7 (WG1) dQ
+// read-out, one thread per query row; warp 8 MMA issuer; warp 9 TMA producer;
+// warps 10-11 idle.  No register split: 384 threads leave 168 registers each.
+
+constexpr int kBwdThreads = 384;
+
+enum BwdBar {
+  BB_KV = 0,        // K and V tiles of this CTA landed (TMA tx)
+  BB_QFULL = 1,     // [2] Q tile + its LSE / D rows landed (32 producer lanes + TMA tx)
+  BB_QFREE = 3,     // [2] Q slot free: its last MMA (dK) completed
+  BB_OFULL = 5,     // [2] dO tile landed (TMA tx)
+  BB_OFREE = 7,     // [2] dO slot free: its last MMA (dV) completed
+  BB_SDP = 9,       // S^T and dP^T complete
+  BB_PDS = 10,      // P^T, dS^T in tensor memory and dS in shared memory (128 WG0 threads)
+  BB_DQ = 11,       // dQ tile complete
+  BB_DQFREE = 12,   // dQ tile read out (128 WG1 threads)
+  BB_DONE = 13,     // every MMA complete: dK, dV final
+  BB_COUNT = 14,
+};
+
+template <int D>
+struct BCfg {
+  static constexpr int kTileBytes = kBlockM * D * 2;  // 128 rows x d bf16
+  static constexpr int kChunks = D / 64;
+  static constexpr int kOStages = (D == 128) ? 1 : 2;  // shared memory budget at d = 128
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kTileBytes;
+  static constexpr int kOffQ = kOffV + kTileBytes;                 // [2]
+  static constexpr int kOffO = kOffQ + 2 * kTileBytes;             // [kOStages]
+  static constexpr int kOffDS = kOffO + kOStages * kTileBytes;     // 128 keys x 128 queries bf16
+  static constexpr int kOffLse = kOffDS + kBlockN * kBlockM * 2;   // [2][128] log2-domain LSE
+  static constexpr int kOffDelta = kOffLse + 2 * kBlockM * 4;      // [2][128] D_i
+  static constexpr int kOffBar = kOffDelta + 2 * kBlockM * 4;
+  static constexpr int kOffMisc = kOffBar + BB_COUNT * 8;
+  static constexpr int kUsed = kOffMisc + 16;
+  static constexpr int kSmemBytes = kUsed + 1024;
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kColDK + D <= 512, "TMEM budget");
+};
+
+struct BwdParams {
+  const float* lse2;    // [B, Hq, Nq] LSE * log2 e (+inf for a row with no visible key)
+  const float* delta;   // [B, Hq, Nq] D_i
+  float* dq_acc;        // [B, Nq, Hq, d] fp32, zero before the main kernel
+  __nv_bfloat16* dk;    // [B, Nk, Hkv, d]
+  __nv_bfloat16* dv;    // [B, Nk, Hkv, d]
+  int B, Hq, Hkv, Nq, Nk;
+  int wl, wr;
+  float scale;
+  float c;              // scale * log2 e (any sign)
+  uint32_t limit_ns;
+};
+
+// Query tiles [lo, hi] whose rows see any key of key block kb (hi < lo: none).
+__host__ __device__ inline void query_tiles_for(const BwdParams& p, int kb, int& lo, int& hi) {
+  const int koff = p.Nk - p.Nq;
+  const int k0 = kb * kBlockN;
+  const int k1 = (k0 + kBlockN - 1 < p.Nk - 1) ? k0 + kBlockN - 1 : p.Nk - 1;
+  int first = (p.wr >= 0) ? k0 - p.wr - koff : 0;      // g_i + wr >= k0
+  int last = (p.wl >= 0) ? k1 + p.wl - koff : p.Nq - 1;  // g_i - wl <= k1
+  if (first < 0) first = 0;
+  if (last > p.Nq - 1) last = p.Nq - 1;
+  if (first > last) {
+    lo = 0;
+    hi = -1;
+    return;
+  }
+  lo = first / kBlockM;
+  hi = last / kBlockM;
+}
+
+// D_i = dO_i . O_i and the log2-domain LSE; zeroes the dQ accumulator.
+// One warp per (batch, head, row); lanes split d.
+template <int D>
+__global__ void __launch_bounds__(256) fa2_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
+                                                           const __nv_bfloat16* __restrict__ dout,
+                                                           const float* __restrict__ lse,
+                                                           float* lse2, float* delta, float* dq_acc,
+                                                           int B, int Hq, int Nq) {
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= static_cast<long long>(B) * Nq * Hq) return;
+  // row enumerates [B, Nq, Hq] (the layout of o and dout)
+  const int hq = static_cast<int>(row % Hq);
+  const long long bi = row / Hq;
+  const int i = static_cast<int>(bi % Nq), b = static_cast<int>(bi / Nq);
+  const __nv_bfloat16* orow = o + row * D;
+  const __nv_bfloat16* grow = dout + row * D;
+  float acc = 0.f;
+  for (int c = lane; c < D; c += 32) acc = fmaf(__bfloat162float(orow[c]), __bfloat162float(grow[c]), acc);
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  float* qrow = dq_acc + row * D;
+  for (int c = lane; c < D; c += 32) qrow[c] = 0.f;
+  if (lane == 0) {
+    const long long s = (static_cast<long long>(b) * Hq + hq) * Nq + i;
+    const float l = lse[s];
+    delta[s] = acc;
+    lse2[s] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+  }
+}
+
+// dQ = bf16(dQ accumulator).
+__global__ void __launch_bounds__(256) fa2_bwd_dq_kernel(const float* __restrict__ dq_acc,
+                                                         __nv_bfloat16* dq, long long n4) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= n4) return;
+  const float4 v = reinterpret_cast<const float4*>(dq_acc)[idx];
+  uint2 w;
+  w.x = pack_bf16x2(v.x, v.y);
+  w.y = pack_bf16x2(v.z, v.w);
+  reinterpret_cast<uint2*>(dq)[idx] = w;
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const BwdParams p) {
+  using C = BCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t bar0 = sbase + C::kOffBar;
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
+  float* sm_lse = reinterpret_cast<float*>(smem + C::kOffLse);
+  float* sm_delta = reinterpret_cast<float*>(smem + C::kOffDelta);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int kb = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int group = p.Hq / p.Hkv;
+  const int koff = p.Nk - p.Nq;
+  int qt_lo, qt_hi;
+  query_tiles_for(p, kb, qt_lo, qt_hi);
+  const int n_qt = qt_hi - qt_lo + 1 > 0 ? qt_hi - qt_lo + 1 : 0;
+  const int n_it = n_qt * group;  // iteration it: head hk*group + it / n_qt, query tile qt_lo + it % n_qt
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < BB_COUNT; ++i) {
+      uint32_t cnt = 1;
+      if (i == BB_QFULL || i == BB_QFULL + 1) cnt = 32;
+      if (i == BB_PDS || i == BB_DQFREE) cnt = kBlockM;
+      mbar_init(bar(i), cnt);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 9 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitGuard g{smem_addr(const_cast<int*>(abort_flag)), p.limit_ns};
+
+  if (warp < 4) {
+    // ============ WG0: P^T and dS^T, one thread per key row ============
+    const int kr = warp * 32 + lane;          // key row in the block == TMEM lane
+    const int key = kb * kBlockN + kr;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::kColS, tDP = tmem + lane_off + C::kColDP;
+    const uint32_t sDS = sbase + C::kOffDS;
+    bool ok = true;
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int st = it & 1;
+      const int qt = qt_lo + it % n_qt;
+      const int q0 = qt * kBlockM;
+      if (!mbar_wait_warp(bar(BB_SDP), it & 1, g, FA2_SITE_S_READY, it)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // visible query columns of this key row: g_i - wl <= key <= g_i + wr
+      // (a tile needs masking when some key lies right of some row's right
+      // bound, left of some row's left bound, or past the sequences' ends)
+      const int k0 = kb * kBlockN;
+      const bool masked = (q0 + kBlockM > p.Nq) || (k0 + kBlockN > p.Nk) ||
+                          (p.wr >= 0 && k0 + kBlockN - 1 > q0 + koff + p.wr) ||
+                          (p.wl >= 0 && k0 < q0 + kBlockM - 1 + koff - p.wl);
+      const float* lse_s = sm_lse + st * kBlockM;
+      const float* dl_s = sm_delta + st * kBlockM;
+#pragma unroll 1
+      for (int ch = 0; ch < kBlockM / 32; ++ch) {
+        uint32_t rs[32], rd[32];
+        tmem_ld32(tS + 32 * ch, rs);
+        tmem_ld32(tDP + 32 * ch, rd);
+        tmem_wait_ld();
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int qc = 32 * ch + 2 * i + e;  // query column in the tile
+            float pe = ex2_approx(fmaf(__uint_as_float(rs[2 * i + e]), p.c, -lse_s[qc]));
+            if (masked) {
+              const int gi = q0 + qc + koff;  // diagonal key of query row q0 + qc
+              const bool vis = (q0 + qc < p.Nq) && (key < p.Nk) && (p.wl < 0 || key >= gi - p.wl) &&
+                               (p.wr < 0 || key <= gi + p.wr);
+              if (!vis) pe = 0.f;
+            }
+            pv[e] = pe;
+            dsv[e] = pe * (__uint_as_float(rd[2 * i + e]) - dl_s[qc]);
+          }
+          pk[i] = pack_bf16x2(pv[0], pv[1]);
+          dk[i] = pack_bf16x2(dsv[0], dsv[1]);
+        }
+        // bf16 P^T / dS^T over the S^T / dP^T columns this loop has consumed
+        tmem_st16(tS + 16 * ch, pk);
+        tmem_st16(tDP + 16 * ch, dk);
+        // dS^T row into shared memory: queries [32 ch, 32 ch + 32) of key row
+        // kr, MN-major SW128 (query chunk of 64 = 16 KiB block, 128 B per key)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int q8 = 32 * ch + 8 * u;  // first of 8 queries in this 16-byte unit
+          const int blk = q8 / 64, unit = (q8 % 64) / 8;
+          const uint32_t addr = sDS + blk * (kBlockN * 128) + kr * 128 + ((unit ^ (kr & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dk[4 * u]),
+                       "r"(dk[4 * u + 1]), "r"(dk[4 * u + 2]), "r"(dk[4 * u + 3])
+                       : "memory");
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(BB_PDS));
+    }
+    // ---- epilogue: dK (scaled) and dV rows of this key block ----
+    if (ok && n_it > 0 && !mbar_wait_warp(bar(BB_DONE), 0, g, FA2_SITE_MMA_DRAIN, 0)) ok = false;
+    tc_fence_after();
+    // (the TMEM loads run on the whole warp -- tcgen05.ld is warp-collective --
+    // and only the stores are limited to keys inside the sequence)
+    const bool valid = key < p.Nk;
+    if (ok) {
+      const size_t row = ((static_cast<size_t>(b) * p.Nk + (valid ? key : 0)) * p.Hkv + hk) * D;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tcol = tmem + lane_off + (which ? C::kColDK : C::kColDV);
+        const float mul = which ? p.scale : 1.f;
+        __nv_bfloat16* dst = (which ? p.dk : p.dv) + row;
+#pragma unroll 1
+        for (int ch = 0; ch < D / 16; ++ch) {
+          uint32_t r[16];
+          if (n_it > 0) {
+            tmem_ld16(tcol + 16 * ch, r);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) r[i] = 0u;
+          }
+          uint4 w0, w1;
+          w0.x = pack_bf16x2(__uint_as_float(r[0]) * mul, __uint_as_float(r[1]) * mul);
+          w0.y = pack_bf16x2(__uint_as_float(r[2]) * mul, __uint_as_float(r[3]) * mul);
+          w0.z = pack_bf16x2(__uint_as_float(r[4]) * mul, __uint_as_float(r[5]) * mul);
+          w0.w = pack_bf16x2(__uint_as_float(r[6]) * mul, __uint_as_float(r[7]) * mul);
+          w1.x = pack_bf16x2(__uint_as_float(r[8]) * mul, __uint_as_float(r[9]) * mul);
+          w1.y = pack_bf16x2(__uint_as_float(r[10]) * mul, __uint_as_float(r[11]) * mul);
+          w1.z = pack_bf16x2(__uint_as_float(r[12]) * mul, __uint_as_float(r[13]) * mul);
+          w1.w = pack_bf16x2(__uint_as_float(r[14]) * mul, __uint_as_float(r[15]) * mul);
+          if (valid) {
+            reinterpret_cast<uint4*>(dst + 16 * ch)[0] = w0;
+            reinterpret_cast<uint4*>(dst + 16 * ch)[1] = w1;
+          }
+        }
+      }
+    }
+  } else if (warp < 8) {
+    // ============ WG1: dQ read-out, one thread per query row ============
+    const int qr = (warp - 4) * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    const uint32_t tQ = tmem + lane_off + C::kColS;
+    for (int it = 0; it < n_it; ++it) {
+      const int hq = hk * group + it / n_qt;
+      const int row = (qt_lo + it % n_qt) * kBlockM + qr;
+      if (!mbar_wait_warp(bar(BB_DQ), it & 1, g, FA2_SITE_O_FINAL, it)) break;
+      tc_fence_after();
+      float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.Nq + row) * p.Hq + hq) * D;
+#pragma unroll 1
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t r[32];
+        tmem_ld32(tQ + 32 * ch, r);
+        tmem_wait_ld();
+        if (row < p.Nq) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            red_add_v4(dst + 32 * ch + 4 * i, __uint_as_float(r[4 * i]) * p.scale,
+                       __uint_as_float(r[4 * i + 1]) * p.scale, __uint_as_float(r[4 * i + 2]) * p.scale,
+                       __uint_as_float(r[4 * i + 3]) * p.scale);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(BB_DQFREE));
+    }
+  } else if (warp == 8) {
+    // ============ MMA issuer ============
+    const uint32_t sK = sbase + C::kOffK, sV = sbase + C::kOffV;
+    const uint32_t idSS = idesc_bf16_f32_ab(kBlockN, kBlockM, false, false);  // S^T, dP^T: K-major A and B
+    const uint32_t idTS = idesc_bf16_f32_ab(kBlockN, D, false, true);         // dV, dK: B (dO, Q) MN-major
+    const uint32_t idDQ = idesc_bf16_f32_ab(kBlockM, D, true, true);          // dQ: A (dS) and B (K) MN-major
+    const uint64_t dK_k = sw128_desc(sK, 16, 1024), dV_k = sw128_desc(sV, 16, 1024);
+    const uint64_t dK_mn = sw128_desc(sK, kChunkBytes, 1024);
+    const uint64_t dDS = sw128_desc(sbase + C::kOffDS, kBlockN * 128, 1024);
+    auto commit = [&](uint32_t bb) {
+      if (elect_one()) umma_commit(bb);
+      __syncwarp();
+    };
+    bool ok = n_it > 0 && mbar_wait_warp(bar(BB_KV), 0, g, FA2_SITE_KV_LOADED, 0);
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int qs = it & 1, os = it % C::kOStages;
+      if (!mbar_wait_warp(bar(BB_QFULL + qs), (it >> 1) & 1, g, FA2_SITE_Q_LOADED, it) ||
+          !mbar_wait_warp(bar(BB_OFULL + os), (it / C::kOStages) & 1, g, FA2_SITE_Q_LOADED, it) ||
+          (it > 0 && !mbar_wait_warp(bar(BB_DQFREE), (it - 1) & 1, g, FA2_SITE_O_RESCALED, it))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t sQ = sbase + C::kOffQ + qs * C::kTileBytes;
+      const uint32_t sO = sbase + C::kOffO + os * C::kTileBytes;
+      uint64_t aK = dK_k, aV = dV_k, bQ = sw128_desc(sQ, 16, 1024), bO = sw128_desc(sO, 16, 1024);
+      asm volatile("" : "+l"(aK), "+l"(aV), "+l"(bQ), "+l"(bO));
+      if (elect_one()) {
+        // S^T = K Q^T and dP^T = V dO^T: K advances 32 B in a swizzle atom,
+        // then jumps to the next 64-column chunk
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t step = ((kk & 3) == 3) ? (kChunkBytes - 3 * 32) >> 4 : 32 >> 4;
+          umma_ss(tmem + C::kColS, aK, bQ, idSS, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + C::kColDP, aV, bO, idSS, kk > 0 ? 1u : 0u);
+          aK += step;
+          aV += step;
+          bQ += step;
+          bO += step;
+        }
+        umma_commit(bar(BB_SDP));
+      }
+      __syncwarp();
+      if (!mbar_wait_warp(bar(BB_PDS), it & 1, g, FA2_SITE_P_READY, it)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint64_t bOm = sw128_desc(sO, kChunkBytes, 1024), bQm = sw128_desc(sQ, kChunkBytes, 1024);
+      uint64_t aDS = dDS, bKm = dK_mn;
+      asm volatile("" : "+l"(bOm), "+l"(bQm), "+l"(aDS), "+l"(bKm));
+      if (elect_one()) {
+        // dV += P^T dO and dK += dS^T Q: A from TMEM (8 columns per 16 queries),
+        // B MN-major (16 query rows = 2 KiB per step)
+#pragma unroll
+        for (int kk = 0; kk < kBlockM / 16; ++kk) {
+          umma_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8, bOm, idTS, (it > 0 || kk > 0) ? 1u : 0u);
+          bOm += (16 * kSwizzleBytes) >> 4;
+        }
+        umma_commit(bar(BB_OFREE + os));
+#pragma unroll
+        for (int kk = 0; kk < kBlockM / 16; ++kk) {
+          umma_ts(tmem + C::kColDK, tmem + C::kColDP + kk * 8, bQm, idTS, (it > 0 || kk > 0) ? 1u : 0u);
+          bQm += (16 * kSwizzleBytes) >> 4;
+        }
+        umma_commit(bar(BB_QFREE + qs));
+        // dQ tile = dS K: A = dS (queries x keys, MN-major in shared memory),
+        // B = K (keys x d, MN-major); 16 keys = 2 KiB per step in both
+#pragma unroll
+        for (int kk = 0; kk < kBlockN / 16; ++kk) {
+          umma_ss(tmem + C::kColS, aDS, bKm, idDQ, kk > 0 ? 1u : 0u);
+          aDS += (16 * kSwizzleBytes) >> 4;
+          bKm += (16 * kSwizzleBytes) >> 4;
+        }
+        umma_commit(bar(BB_DQ));
+      }
+      __syncwarp();
+    }
+    // drain: every MMA complete before dK / dV are read and TMEM is freed
+    const WaitGuard drain{0u, p.limit_ns};
+    if (n_it > 0) {
+      commit(bar(BB_DONE));
+      mbar_wait_warp(bar(BB_DONE), 0, drain, FA2_SITE_MMA_DRAIN, 0);
+    }
+  } else if (warp == 9) {
+    // ============ TMA producer ============
+    bool ok = n_it > 0;
+    if (ok) {
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar(BB_KV), 2 * C::kTileBytes);
+#pragma unroll
+        for (int ch = 0; ch < C::kChunks; ++ch) {
+          tma_load_4d(sbase + C::kOffK + ch * kChunkBytes, &tmK, bar(BB_KV), ch * 64, hk, kb * kBlockN, b);
+          tma_load_4d(sbase + C::kOffV + ch * kChunkBytes, &tmV, bar(BB_KV), ch * 64, hk, kb * kBlockN, b);
+        }
+      }
+      __syncwarp();
+    }
+    int it = 0;
+    for (; it < n_it && ok; ++it) {
+      const int qs = it & 1, os = it % C::kOStages;
+      const int hq = hk * group + it / n_qt;
+      const int q0 = (qt_lo + it % n_qt) * kBlockM;
+      if (it >= 2 && !mbar_wait_warp(bar(BB_QFREE + qs), ((it >> 1) - 1) & 1, g, FA2_SITE_KV_FREE, it)) {
+        ok = false;
+        break;
+      }
+      // LSE (log2 domain) and D of the tile's rows; rows past Nq see nothing
+      const size_t srow = (static_cast<size_t>(b) * p.Hq + hq) * p.Nq;
+#pragma unroll
+      for (int e = 0; e < kBlockM / 32; ++e) {
+        const int r = e * 32 + lane, i = q0 + r;
+        sm_lse[qs * kBlockM + r] = (i < p.Nq) ? p.lse2[srow + i] : INFINITY;
+        sm_delta[qs * kBlockM + r] = (i < p.Nq) ? p.delta[srow + i] : 0.f;
+      }
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar(BB_QFULL + qs), C::kTileBytes);
+#pragma unroll
+        for (int ch = 0; ch < C::kChunks; ++ch)
+          tma_load_4d(sbase + C::kOffQ + qs * C::kTileBytes + ch * kChunkBytes, &tmQ, bar(BB_QFULL + qs),
+                      ch * 64, hq, q0, b);
+      } else {
+        mbar_arrive(bar(BB_QFULL + qs));
+      }
+      __syncwarp();
+      if (it >= C::kOStages &&
+          !mbar_wait_warp(bar(BB_OFREE + os), ((it / C::kOStages) - 1) & 1, g, FA2_SITE_KV_FREE, it)) {
+        ok = false;
+        break;
+      }
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar(BB_OFULL + os), C::kTileBytes);
+#pragma unroll
+        for (int ch = 0; ch < C::kChunks; ++ch)
+          tma_load_4d(sbase + C::kOffO + os * C::kTileBytes + ch * kChunkBytes, &tmO, bar(BB_OFULL + os),
+                      ch * 64, hq, q0, b);
+      }
+      __syncwarp();
+    }
+    if (!ok && n_it > 0) {
+      // let the copies in flight land before the CTA exits
+      const WaitGuard drain{0u, p.limit_ns};
+      mbar_wait_warp(bar(BB_KV), 0, drain, FA2_SITE_LOAD_DRAIN, 0);
+      for (int j = (it > 2 ? it - 2 : 0); j < it; ++j) {
+        mbar_wait_warp(bar(BB_QFULL + (j & 1)), (j >> 1) & 1, drain, FA2_SITE_LOAD_DRAIN, j);
+        mbar_wait_warp(bar(BB_OFULL + j % C::kOStages), (j / C::kOStages) & 1, drain, FA2_SITE_LOAD_DRAIN, j);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}

@@ -1253,6 +1253,65 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
   return FA2_OK;
 }
 
+#include "fa2_backward.cuh"
+
+template <int D>
+static int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                      const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+                      int Nk, Window win, float scale, void* workspace, cudaStream_t stream) {
+  using C = BCfg<D>;
+  static std::once_flag once;
+  static int setup_status = FA2_OK;
+  std::call_once(once, [] {
+    if (cudaFuncSetAttribute(fa2_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess)
+      setup_status = FA2_ERR_LAUNCH;
+  });
+  if (setup_status != FA2_OK) return setup_status;
+  const long long rows = static_cast<long long>(B) * Nq * Hq;
+  float* dq_acc = static_cast<float*>(workspace);
+  float* lse2 = dq_acc + ((rows * D + 63) / 64) * 64;
+  float* delta = lse2 + ((rows + 63) / 64) * 64;
+  fa2_bwd_prep_kernel<D><<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
+      dq_acc, B, Hq, Nq);
+  if (cudaGetLastError() != cudaSuccess) return FA2_ERR_LAUNCH;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_bnhd(&tq, q, B, Nq, Hq, D) || !encode_bnhd(&tk, k, B, Nk, Hkv, D) ||
+      !encode_bnhd(&tv, v, B, Nk, Hkv, D) || !encode_bnhd(&tdo, dout, B, Nq, Hq, D))
+    return FA2_ERR_LAUNCH;
+  BwdParams p;
+  p.lse2 = lse2;
+  p.delta = delta;
+  p.dq_acc = dq_acc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.wl = win.wl;
+  p.wr = win.wr;
+  p.scale = scale;
+  p.c = scale * 1.4426950408889634f;
+  p.limit_ns = 1000000000u;
+  const dim3 grid(static_cast<unsigned>((Nk + kBlockN - 1) / kBlockN), Hkv, B);
+  fa2_bwd_kernel<D><<<grid, kBwdThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
+  if (cudaGetLastError() != cudaSuccess) return FA2_ERR_LAUNCH;
+  const long long n4 = rows * D / 4;
+  fa2_bwd_dq_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(
+      dq_acc, static_cast<__nv_bfloat16*>(dq), n4);
+  return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_LAUNCH;
+}
+
+// Bytes of backward workspace: the fp32 dQ accumulator, then LSE in log2
+// units and D per row (each region rounded up to 64 floats).
+static long long bwd_workspace_bytes(int B, int Hq, int Nq, int d) {
+  const long long rows = static_cast<long long>(B) * Nq * Hq;
+  return 4LL * (((rows * d + 63) / 64) * 64 + 2 * ((rows + 63) / 64) * 64);
+}
+
 static int check_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA2_ERR_DEVICE;
@@ -1365,6 +1424,38 @@ extern "C" int fa2_forward_static_ws(const void* q, const void* k, const void* v
   // a problem whose plan needs more than the array is refused (FA2_ERR_WORKSPACE)
   return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal_window(causal), softmax_scale,
                       scratch, static_cast<long long>(kStaticScratchBytes), stream);
+}
+
+extern "C" long long fa2_backward_workspace_size(int B, int Hq, int Nq, int d) {
+  if (B <= 0 || Hq <= 0 || Nq <= 0 || (d != 64 && d != 128)) return -1;
+  return bwd_workspace_bytes(B, Hq, Nq, d);
+}
+
+extern "C" int fa2_backward(const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                            int Hq, int Hkv, int Nq, int Nk, int d, int causal, float softmax_scale,
+                            void* workspace, long long workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
+    return FA2_ERR_NULL_POINTER;
+  const int sv = validate_shape(B, Hq, Hkv, Nq, Nk, d);
+  if (sv != FA2_OK) return sv;
+  if (Hkv > 65535 || B > 65535) return FA2_ERR_SIZE;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
+       reinterpret_cast<uintptr_t>(o) | reinterpret_cast<uintptr_t>(dout) | reinterpret_cast<uintptr_t>(dq) |
+       reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv) |
+       reinterpret_cast<uintptr_t>(workspace)) & 15u)
+    return FA2_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return FA2_ERR_ALIGNMENT;
+  if (!std::isfinite(softmax_scale)) return FA2_ERR_SCALE;
+  if (workspace_bytes < bwd_workspace_bytes(B, Hq, Nq, d)) return FA2_ERR_WORKSPACE;
+  const int dv_ = check_device();
+  if (dv_ != FA2_OK) return dv_;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, causal_window(causal),
+                           softmax_scale, workspace, s);
+  return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, causal_window(causal),
+                        softmax_scale, workspace, s);
 }
 
 extern "C" long long fa2_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal) {

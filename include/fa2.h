@@ -184,6 +184,41 @@ int fa2_forward_static_ws(const void* q, const void* k, const void* v, void* o, 
                           float softmax_scale, void* stream);
 #define FA2_STATIC_WS_BYTES (40LL << 20)
 
+/*
+ * fa2_backward -- gradients of the forward pass: given q, k, v, the forward's
+ * o and lse, and an upstream gradient dout (bf16 [B, Nq, Hq, d], like o),
+ * writes dq (bf16 [B, Nq, Hq, d]), dk and dv (bf16 [B, Nk, Hkv, d]):
+ *
+ *   P_ij = exp(softmax_scale q_i . k_j - lse_i) over the keys row i sees
+ *   D_i  = dout_i . o_i,  dS_ij = P_ij (dout_i . v_j - D_i)
+ *   dq_i = softmax_scale sum_j dS_ij k_j,  dk_j = softmax_scale sum_i dS_ij q_i,
+ *   dv_j = sum_i P_ij dout_i    (dk, dv summed over each KV head's query group)
+ *
+ * the chain rule on the forward's definition, with P recomputed tile by tile
+ * from lse so nothing of size Nq x Nk is stored; the pages report the
+ * forward+backward figures of the method ("FlashAttention 2: Three Places the
+ * Chip Was Still Waiting", section 2.5).  Three kernels on `stream`: D and
+ * the log2 LSE per row (and zeroing of the dq accumulator), the main kernel
+ * (one block per 128-key block, KV head and batch, tcgen05 MMAs, dq summed
+ * with fp32 vector atomics), and the bf16 rounding of dq.
+ *
+ *   workspace        device pointer, 16-byte aligned, at least
+ *                    fa2_backward_workspace_size(B, Hq, Nq, d) bytes of
+ *                    scratch: the fp32 dq accumulator and two floats per row
+ *   causal, softmax_scale, sizes: as the forward call that produced o, lse
+ *
+ * Returns the fa2_forward codes, FA2_ERR_WORKSPACE for a short workspace and
+ * FA2_ERR_SIZE when Hkv or B exceeds 65535.  Rows with no visible key
+ * (lse = -inf) get dq = 0 and contribute nothing.
+ */
+int fa2_backward(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+                 int Nk, int d, int causal, float softmax_scale, void* workspace,
+                 long long workspace_bytes, void* stream);
+
+/* Bytes of scratch fa2_backward needs (-1 for invalid arguments). */
+long long fa2_backward_workspace_size(int B, int Hq, int Nq, int d);
+
 /* Human-readable text for a status code (static storage, never NULL). */
 const char* fa2_status_string(int status);
 

@@ -1,0 +1,74 @@
+"""Backward pass on the GPU vs the fp64 oracle (gradients from the definition).
+
+Tolerance, derived from the arithmetic: P and dS enter the tensor cores as
+bf16 (relative rounding 2^-9), are accumulated in fp32, and dS also carries
+the forward's bf16 O through D = dO . O.  Each gradient is compared relative
+to its own scale: max |err| <= 3e-2 * max |ref| and mean |err| <= 1e-2 *
+mean |ref|, with no NaN or Inf.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_tiled_attention_29_b200.inputs import Workload, bf16_bits, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+MAX_REL, MEAN_REL = 3e-2, 1e-2
+
+
+@pytest.fixture(scope="module")
+def fa2():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import exact_tiled_attention_29_b200 as m
+    return m
+
+
+def grads_gpu(fa2, q, k, v, g, causal, scale):
+    dev = torch.device("cuda")
+    qd, kd, vd, gd = (t.to(dev) for t in (q, k, v, g))
+    o, lse = fa2.attention(qd, kd, vd, causal=causal, softmax_scale=scale)
+    dq, dk, dv = fa2.attention_backward(qd, kd, vd, o, lse, gd, causal=causal, softmax_scale=scale)
+    torch.cuda.synchronize()
+    assert fa2.fa2_debug_status(None) == 0
+    return [t.float().cpu().numpy() for t in (dq, dk, dv)]
+
+
+def check(fa2, w, scale=None):
+    q, k, v = make_qkv(w)
+    g = torch.randn(q.shape, generator=torch.Generator().manual_seed(w.seed + 99)).to(torch.bfloat16)
+    scale = w.softmax_scale if scale is None else scale
+    got = grads_gpu(fa2, q, k, v, g, w.causal, scale)
+    ref = oracle.backward(bf16_bits(q), bf16_bits(k), bf16_bits(v), bf16_bits(g), w.causal, scale)
+    for name, a, r in zip(("dQ", "dK", "dV"), got, ref):
+        assert np.isfinite(a).all(), f"{w.name}: non-finite {name}"
+        err = np.abs(a - r)
+        big = max(np.abs(r).max(), 1e-6)
+        assert err.max() <= MAX_REL * big, f"{w.name} {name}: max err {err.max():.3g} vs scale {big:.3g}"
+        assert err.mean() <= MEAN_REL * max(np.abs(r).mean(), 1e-9), \
+            f"{w.name} {name}: mean err {err.mean():.3g} vs mean {np.abs(r).mean():.3g}"
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("nq,nk", [(256, 256), (300, 300), (129, 700), (700, 129), (1, 200), (1000, 1000)])
+def test_backward_vs_oracle(fa2, d, causal, nq, nk):
+    check(fa2, Workload(f"bwd{nq}x{nk}", 2, 4, 2, nq, nk, d, causal, seed=nq * 5 + nk + d))
+
+
+def test_backward_gqa_and_scale(fa2):
+    check(fa2, Workload("bwd_gqa", 1, 8, 2, 512, 512, 128, True, seed=51), scale=0.2)
+    check(fa2, Workload("bwd_neg", 1, 2, 2, 384, 384, 64, False, seed=52), scale=-0.1)
+
+
+def test_backward_deterministic_dk_dv(fa2):
+    # dK and dV are summed in tensor memory in a fixed order: bitwise repeatable
+    w = Workload("bwd_det", 2, 4, 2, 640, 640, 128, True, seed=53)
+    q, k, v = make_qkv(w)
+    g = torch.randn(q.shape, generator=torch.Generator().manual_seed(54)).to(torch.bfloat16)
+    a = grads_gpu(fa2, q, k, v, g, True, w.softmax_scale)
+    b = grads_gpu(fa2, q, k, v, g, True, w.softmax_scale)
+    assert np.array_equal(a[1], b[1]) and np.array_equal(a[2], b[2])

@@ -66,6 +66,22 @@ def test_local_window_validation():
     assert fa2.fa2_forward_local(16, 32, 48, 64, 80, 1, 2, 1, 5, 7, 80, 3, 0, 0.1, None) == 3
 
 
+def test_backward_validation():
+    ok = dict(q=16, k=32, v=48, o=64, lse=80, dout=96, dq=112, dk=128, dv=144, B=1, Hq=2, Hkv=1,
+              Nq=5, Nk=7, d=128, causal=1, scale=0.1, ws=160, wsb=1 << 20)
+
+    def call(**over):
+        a = dict(ok, **over)
+        return fa2.fa2_backward(a["q"], a["k"], a["v"], a["o"], a["lse"], a["dout"], a["dq"], a["dk"],
+                                a["dv"], a["B"], a["Hq"], a["Hkv"], a["Nq"], a["Nk"], a["d"],
+                                a["causal"], a["scale"], a["ws"], a["wsb"], None)
+    assert call(dout=0) == 1 and call(ws=0) == 1
+    assert call(Hq=3, Hkv=2) == 2 and call(d=96) == 3 and call(dq=120) == 4 and call(lse=81) == 4
+    assert call(scale=math.inf) == 5 and call(wsb=16) == 10
+    assert fa2.fa2_backward_workspace_size(1, 2, 5, 128) >= 4 * 5 * 2 * 128
+    assert fa2.fa2_backward_workspace_size(1, 2, 5, 80) == -1
+
+
 def test_valid_arguments_reach_the_device_check_only():
     import torch
     st = call()

@@ -55,6 +55,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--direction", default="fwd", choices=["fwd", "bwd"],
+                    help="fwd: the forward pass (the headline); bwd: fa2_backward on the forward's "
+                         "outputs, FLOPs counted as 2.5x the forward's (five matrix products "
+                         "instead of two)")
     ap.add_argument("--schedule", default="units", choices=["units", "streamk"],
                     help="streamk: fa2_forward_ws, one persistent block per SM over a workspace; "
                          "units: fa2_forward, one block per (query block, head, batch)")
@@ -445,11 +449,119 @@ def run_fa2(args, w):
     return 0
 
 
+def run_fa2_backward(args, w):
+    """Times fa2_backward (its three kernels) on one GPU; same timing rules as the forward."""
+    import torch
+    import exact_tiled_attention_29_b200 as fa2
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1 or w.windowed:
+        raise SystemExit("--direction bwd runs on one GPU, without a window")
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    q_h, k_h, v_h = make_qkv(w)
+    g_h = torch.randn(q_h.shape, generator=torch.Generator().manual_seed(w.seed + 7)).to(torch.bfloat16)
+    q, k, v, g = (t.to(dev) for t in (q_h, k_h, v_h, g_h))
+    stream = torch.cuda.current_stream(dev)
+    o, lse = fa2.attention(q, k, v, causal=w.causal, softmax_scale=w.softmax_scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa2.fa2_backward_workspace_size(w.B, w.Hq, w.Nq, w.d), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(qq, kk, vv, oo, ll, gg, a, b_, c):
+        st = fa2.fa2_backward(qq, kk, vv, oo, ll, gg, a, b_, c, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d,
+                              w.causal, w.softmax_scale, ws, ws.numel(), stream)
+        if st != 0:
+            raise fa2.FA2Error(st, "fa2_backward")
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step(q, k, v, o, lse, g, dq, dk, dv)
+    torch.cuda.synchronize()
+    if fa2.fa2_debug_status(stream) != 0:
+        raise RuntimeError("device status after warm-up")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step(q, k, v, o, lse, g, dq, dk, dv)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    mean_ms = sum(s_.elapsed_time(e) for s_, e in zip(starts, ends)) / args.steps
+    if fa2.fa2_debug_status(stream) != 0:
+        raise RuntimeError("device status after the timed region")
+    flops = 2.5 * w.flops()
+    e2e = None
+    if not args.no_e2e:
+        hosts = [t.cpu().pin_memory() for t in (q, k, v, o, lse, g)]
+        devs = [torch.empty_like(t) for t in (q, k, v, o, lse, g)]
+        outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+        n_e2e = max(3, min(args.steps, 30))
+
+        def e2e_step():
+            for d_, h_ in zip(devs, hosts):
+                d_.copy_(h_, non_blocking=True)
+            step(*devs, dq, dk, dv)
+            for h_, d_ in zip(outs_h, (dq, dk, dv)):
+                h_.copy_(d_, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / n_e2e
+        e2e = {"value": flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hosts),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs_h),
+               "steps": n_e2e}
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        sub = w.with_(B=1, Hq=w.Hq // w.Hkv, Hkv=1, Nq=min(w.Nq, 1024), Nk=min(w.Nk, 1024))
+        sq, sk, sv = (bf16_bits(t) for t in make_qkv(sub))
+        sg = bf16_bits(torch.randn((sub.B, sub.Nq, sub.Hq, sub.d),
+                                   generator=torch.Generator().manual_seed(1)).to(torch.bfloat16))
+        t0 = time.perf_counter()
+        oracle.backward(sq, sk, sv, sg, sub.causal, sub.softmax_scale)
+        dt = time.perf_counter() - t0
+        cpu = {"value": 2.5 * sub.flops() / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+               "sample": f"backward of one KV-head group (B=1, Hq={sub.Hq}, Hkv=1) at "
+                         f"N={sub.Nq}, d={sub.d}, causal={sub.causal}: fp64 C oracle, one group "
+                         f"per thread; {2.5 * sub.flops():.3g} algorithmic FLOP in {dt:.2f} s"}
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (mean_ms * 1e-3) / 1e12
+    line = {"metric": "attention backward TFLOP/s (2.5x forward FLOPs)", "value": achieved,
+            "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": mean_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic", "config": {**workload_config(w, 1), "direction": "bwd"},
+            "pct_of_peak": 100.0 * achieved / peak,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"bf16_tflops (burst), {peak_src}",
+                         "kernel": f"fa2_bwd_kernel<{w.d}> + prep + dq rounding (timed together)"},
+            "gpu_launches": 3 * args.steps, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
+            "kernel_source_sha256_16": kernel_source_hash()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     w = ALL_WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.direction == "bwd":
+        return run_fa2_backward(args, w)
     return run_fa2(args, w)
 
 

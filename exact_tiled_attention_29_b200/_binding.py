@@ -23,7 +23,7 @@ STATUS_NAMES = {
 SITE_NAMES = {
     1: "Q_LOADED", 2: "KV_LOADED", 3: "KV_FREE", 4: "S_READY", 5: "P_READY", 6: "STATS_READY",
     7: "O_RESCALED", 8: "O_FINAL", 9: "FINAL_STATS", 10: "MMA_DRAIN", 11: "LOAD_DRAIN",
-    15: "SELFTEST",
+    13: "SMEM_ALIGN", 15: "SELFTEST",
 }
 FA2_SITE_SELFTEST = 15
 FA2_STATIC_WS_BYTES = 40 << 20  # the library's fixed stream-K scratch per device (fa2.h)

@@ -32,12 +32,13 @@
 //   MMA   dV += P^T dO (TS), dK += dS^T Q (TS), dQ_tile = dS K (SS, into the
 //         S^T columns, after the dV MMA read P^T: one thread's MMAs run in
 //         issue order)                                     -> "dQ ready"
-//   WG1   read dQ_tile, scale, add into the fp32 accumulator -> "dQ free"
+//   WG0/1 read dQ_tile, scale, add into the fp32 accumulator -> "dQ free"
 //   and the next tile's S^T may overwrite the columns.
 //
-// Roles: warps 0-3 (WG0) P / dS, one thread per key row; warps 4-7 (WG1) dQ
-// read-out, one thread per query row; warp 8 MMA issuer; warp 9 TMA producer;
-// warps 10-11 idle.  No register split: 384 threads leave 168 registers each.
+// Roles: warps 0-3 (WG0) and 4-7 (WG1) split the query columns of P / dS
+// (one thread per key row) and of the dQ read-out (one thread per query
+// row); warp 8 MMA issuer; warp 9 TMA producer; warps 10-11 idle.  No
+// register split: 384 threads leave 168 registers each.
 
 constexpr int kBwdThreads = 384;
 
@@ -59,7 +60,7 @@ template <int D>
 struct BCfg {
   static constexpr int kTileBytes = kBlockM * D * 2;  // 128 rows x d bf16
   static constexpr int kChunks = D / 64;
-  static constexpr int kOStages = (D == 128) ? 1 : 2;  // shared memory budget at d = 128
+  static constexpr int kOStages = 2;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kTileBytes;
   static constexpr int kOffQ = kOffV + kTileBytes;                 // [2]
@@ -70,11 +71,18 @@ struct BCfg {
   static constexpr int kOffBar = kOffDelta + 2 * kBlockM * 4;
   static constexpr int kOffMisc = kOffBar + BB_COUNT * 8;
   static constexpr int kUsed = kOffMisc + 16;
-  static constexpr int kSmemBytes = kUsed + 1024;
+  // At d = 128 the tiles leave less than 1 KiB of the 227 KiB for aligning the
+  // base to 1024 bytes; the kernel checks the slack it got (dynamic shared
+  // memory normally starts 1024-aligned, so the slack is 0).
+  static constexpr int kSmemBytes = (kUsed + 1024 < 232448) ? kUsed + 1024 : 232448;
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kColDK + D <= 512, "TMEM budget");
 };
+
+// TMEM column (within the S^T or dP^T block) of the bf16 P^T / dS^T values of
+// query chunk ch (32 queries, 16 columns): 0, 16, 64, 80.
+__host__ __device__ constexpr uint32_t bf16_col(int ch) { return 16u * ch + (ch >= 2 ? 32u : 0u); }
 
 struct BwdParams {
   const float* lse2;    // [B, Hq, Nq] LSE * log2 e (+inf for a row with no visible key)
@@ -165,6 +173,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_addr(smem);
+  if (sbase + C::kUsed > smem_addr(smem_raw) + C::kSmemBytes) {  // uniform: every thread leaves
+    if (threadIdx.x == 0) atomicCAS(&g_status, 0, (FA2_SITE_SMEM_ALIGN << 16) | 1);
+    return;
+  }
   const uint32_t bar0 = sbase + C::kOffBar;
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
   float* sm_lse = reinterpret_cast<float*>(smem + C::kOffLse);
@@ -187,7 +199,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int i = 0; i < BB_COUNT; ++i) {
       uint32_t cnt = 1;
       if (i == BB_QFULL || i == BB_QFULL + 1) cnt = 32;
-      if (i == BB_PDS || i == BB_DQFREE) cnt = kBlockM;
+      if (i == BB_PDS || i == BB_DQFREE) cnt = 2 * kBlockM;
       mbar_init(bar(i), cnt);
     }
     fence_mbar_init();
@@ -208,18 +220,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{smem_addr(const_cast<int*>(abort_flag)), p.limit_ns};
 
-  if (warp < 4) {
-    // ============ WG0: P^T and dS^T, one thread per key row ============
-    const int kr = warp * 32 + lane;          // key row in the block == TMEM lane
+  if (warp < 8) {
+    // ===== WG0 / WG1: P^T and dS^T for query columns [64 wg, 64 wg + 64) of
+    // every key row, then that half of the dQ tile's columns =====
+    const int wg = warp >> 2;
+    const int q4 = warp & 3;
+    const int kr = q4 * 32 + lane;            // key row in the block == TMEM lane (dQ: query row)
     const int key = kb * kBlockN + kr;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::kColS, tDP = tmem + lane_off + C::kColDP;
     const uint32_t sDS = sbase + C::kOffDS;
     bool ok = true;
     for (int it = 0; it < n_it && ok; ++it) {
       const int st = it & 1;
-      const int qt = qt_lo + it % n_qt;
-      const int q0 = qt * kBlockM;
+      const int hq = hk * group + it / n_qt;
+      const int q0 = (qt_lo + it % n_qt) * kBlockM;
       if (!mbar_wait_warp(bar(BB_SDP), it & 1, g, FA2_SITE_S_READY, it)) {
         ok = false;
         break;
@@ -235,19 +250,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float* lse_s = sm_lse + st * kBlockM;
       const float* dl_s = sm_delta + st * kBlockM;
 #pragma unroll 1
-      for (int ch = 0; ch < kBlockM / 32; ++ch) {
+      for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
         uint32_t rs[32], rd[32];
         tmem_ld32(tS + 32 * ch, rs);
         tmem_ld32(tDP + 32 * ch, rd);
         tmem_wait_ld();
         uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float pv[2], dsv[2];
+        for (int i4 = 0; i4 < 8; ++i4) {
+          // log2 LSE and D of 4 query rows (broadcast shared-memory reads)
+          const float4 l4 = reinterpret_cast<const float4*>(lse_s + 32 * ch)[i4];
+          const float4 d4 = reinterpret_cast<const float4*>(dl_s + 32 * ch)[i4];
+          const float lz[4] = {l4.x, l4.y, l4.z, l4.w}, dz[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pv[4], dsv[4];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int qc = 32 * ch + 2 * i + e;  // query column in the tile
-            float pe = ex2_approx(fmaf(__uint_as_float(rs[2 * i + e]), p.c, -lse_s[qc]));
+          for (int e = 0; e < 4; ++e) {
+            const int qc = 32 * ch + 4 * i4 + e;  // query column in the tile
+            float pe = ex2_approx(fmaf(__uint_as_float(rs[4 * i4 + e]), p.c, -lz[e]));
             if (masked) {
               const int gi = q0 + qc + koff;  // diagonal key of query row q0 + qc
               const bool vis = (q0 + qc < p.Nq) && (key < p.Nk) && (p.wl < 0 || key >= gi - p.wl) &&
@@ -255,14 +274,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               if (!vis) pe = 0.f;
             }
             pv[e] = pe;
-            dsv[e] = pe * (__uint_as_float(rd[2 * i + e]) - dl_s[qc]);
+            dsv[e] = pe * (__uint_as_float(rd[4 * i4 + e]) - dz[e]);
           }
-          pk[i] = pack_bf16x2(pv[0], pv[1]);
-          dk[i] = pack_bf16x2(dsv[0], dsv[1]);
+          pk[2 * i4] = pack_bf16x2(pv[0], pv[1]);
+          pk[2 * i4 + 1] = pack_bf16x2(pv[2], pv[3]);
+          dk[2 * i4] = pack_bf16x2(dsv[0], dsv[1]);
+          dk[2 * i4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
-        // bf16 P^T / dS^T over the S^T / dP^T columns this loop has consumed
-        tmem_st16(tS + 16 * ch, pk);
-        tmem_st16(tDP + 16 * ch, dk);
+        // bf16 P^T / dS^T over S^T / dP^T columns this warpgroup has consumed:
+        // chunk ch goes to columns bf16_col(ch) (0, 16, 64, 80), so neither
+        // warpgroup overwrites scores the other has yet to read
+        tmem_st16(tS + bf16_col(ch), pk);
+        tmem_st16(tDP + bf16_col(ch), dk);
         // dS^T row into shared memory: queries [32 ch, 32 ch + 32) of key row
         // kr, MN-major SW128 (query chunk of 64 = 16 KiB block, 128 B per key)
 #pragma unroll
@@ -279,20 +302,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(BB_PDS));
+
+      // ---- this warpgroup's half of the dQ tile (lane = query row) ----
+      if (!mbar_wait_warp(bar(BB_DQ), it & 1, g, FA2_SITE_O_FINAL, it)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int row = q0 + kr;
+      // Read the half row into registers and hand the columns back to the MMA
+      // at once; the atomics then overlap the next tile's products.
+      uint32_t r[D / 2];
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tmem_ld32(tS + wg * (D / 2) + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * c));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(BB_DQFREE));
+      if (row < p.Nq) {
+        float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.Nq + row) * p.Hq + hq) * D + wg * (D / 2);
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i)
+          red_add_v4(dst + 4 * i, __uint_as_float(r[4 * i]) * p.scale, __uint_as_float(r[4 * i + 1]) * p.scale,
+                     __uint_as_float(r[4 * i + 2]) * p.scale, __uint_as_float(r[4 * i + 3]) * p.scale);
+      }
     }
-    // ---- epilogue: dK (scaled) and dV rows of this key block ----
+    // ---- epilogue: WG0 writes dV, WG1 dK (scaled), rows of this key block ----
     if (ok && n_it > 0 && !mbar_wait_warp(bar(BB_DONE), 0, g, FA2_SITE_MMA_DRAIN, 0)) ok = false;
     tc_fence_after();
     // (the TMEM loads run on the whole warp -- tcgen05.ld is warp-collective --
     // and only the stores are limited to keys inside the sequence)
     const bool valid = key < p.Nk;
     if (ok) {
-      const size_t row = ((static_cast<size_t>(b) * p.Nk + (valid ? key : 0)) * p.Hkv + hk) * D;
-#pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
+      const size_t rowk = ((static_cast<size_t>(b) * p.Nk + (valid ? key : 0)) * p.Hkv + hk) * D;
+      const int which = wg;
+      {
         const uint32_t tcol = tmem + lane_off + (which ? C::kColDK : C::kColDV);
         const float mul = which ? p.scale : 1.f;
-        __nv_bfloat16* dst = (which ? p.dk : p.dv) + row;
+        __nv_bfloat16* dst = (which ? p.dk : p.dv) + rowk;
 #pragma unroll 1
         for (int ch = 0; ch < D / 16; ++ch) {
           uint32_t r[16];
@@ -319,33 +366,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
     }
-  } else if (warp < 8) {
-    // ============ WG1: dQ read-out, one thread per query row ============
-    const int qr = (warp - 4) * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
-    const uint32_t tQ = tmem + lane_off + C::kColS;
-    for (int it = 0; it < n_it; ++it) {
-      const int hq = hk * group + it / n_qt;
-      const int row = (qt_lo + it % n_qt) * kBlockM + qr;
-      if (!mbar_wait_warp(bar(BB_DQ), it & 1, g, FA2_SITE_O_FINAL, it)) break;
-      tc_fence_after();
-      float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.Nq + row) * p.Hq + hq) * D;
-#pragma unroll 1
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t r[32];
-        tmem_ld32(tQ + 32 * ch, r);
-        tmem_wait_ld();
-        if (row < p.Nq) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            red_add_v4(dst + 32 * ch + 4 * i, __uint_as_float(r[4 * i]) * p.scale,
-                       __uint_as_float(r[4 * i + 1]) * p.scale, __uint_as_float(r[4 * i + 2]) * p.scale,
-                       __uint_as_float(r[4 * i + 3]) * p.scale);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(bar(BB_DQFREE));
-    }
   } else if (warp == 8) {
     // ============ MMA issuer ============
     const uint32_t sK = sbase + C::kOffK, sV = sbase + C::kOffV;
@@ -360,35 +380,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       __syncwarp();
     };
     bool ok = n_it > 0 && mbar_wait_warp(bar(BB_KV), 0, g, FA2_SITE_KV_LOADED, 0);
-    for (int it = 0; it < n_it && ok; ++it) {
+    // S^T(it) and dP^T(it): dP^T goes first, as soon as Q / dO have landed; S^T
+    // also waits until the previous dQ tile has left the S^T columns.
+    auto issue_s_dp = [&](int it) -> bool {
       const int qs = it & 1, os = it % C::kOStages;
       if (!mbar_wait_warp(bar(BB_QFULL + qs), (it >> 1) & 1, g, FA2_SITE_Q_LOADED, it) ||
-          !mbar_wait_warp(bar(BB_OFULL + os), (it / C::kOStages) & 1, g, FA2_SITE_Q_LOADED, it) ||
-          (it > 0 && !mbar_wait_warp(bar(BB_DQFREE), (it - 1) & 1, g, FA2_SITE_O_RESCALED, it))) {
-        ok = false;
-        break;
-      }
+          !mbar_wait_warp(bar(BB_OFULL + os), (it / C::kOStages) & 1, g, FA2_SITE_Q_LOADED, it))
+        return false;
       tc_fence_after();
       const uint32_t sQ = sbase + C::kOffQ + qs * C::kTileBytes;
       const uint32_t sO = sbase + C::kOffO + os * C::kTileBytes;
       uint64_t aK = dK_k, aV = dV_k, bQ = sw128_desc(sQ, 16, 1024), bO = sw128_desc(sO, 16, 1024);
       asm volatile("" : "+l"(aK), "+l"(aV), "+l"(bQ), "+l"(bO));
+      // K advances 32 B in a swizzle atom, then jumps to the next 64-column chunk
       if (elect_one()) {
-        // S^T = K Q^T and dP^T = V dO^T: K advances 32 B in a swizzle atom,
-        // then jumps to the next 64-column chunk
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t step = ((kk & 3) == 3) ? (kChunkBytes - 3 * 32) >> 4 : 32 >> 4;
-          umma_ss(tmem + C::kColS, aK, bQ, idSS, kk > 0 ? 1u : 0u);
           umma_ss(tmem + C::kColDP, aV, bO, idSS, kk > 0 ? 1u : 0u);
-          aK += step;
+          const uint32_t step = ((kk & 3) == 3) ? (kChunkBytes - 3 * 32) >> 4 : 32 >> 4;
           aV += step;
-          bQ += step;
           bO += step;
+        }
+      }
+      __syncwarp();
+      if (it > 0 && !mbar_wait_warp(bar(BB_DQFREE), (it - 1) & 1, g, FA2_SITE_O_RESCALED, it)) return false;
+      tc_fence_after();
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          umma_ss(tmem + C::kColS, aK, bQ, idSS, kk > 0 ? 1u : 0u);
+          const uint32_t step = ((kk & 3) == 3) ? (kChunkBytes - 3 * 32) >> 4 : 32 >> 4;
+          aK += step;
+          bQ += step;
         }
         umma_commit(bar(BB_SDP));
       }
       __syncwarp();
+      return true;
+    };
+    if (ok) ok = issue_s_dp(0);
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int qs = it & 1, os = it % C::kOStages;
+      const uint32_t sQ = sbase + C::kOffQ + qs * C::kTileBytes;
+      const uint32_t sO = sbase + C::kOffO + os * C::kTileBytes;
       if (!mbar_wait_warp(bar(BB_PDS), it & 1, g, FA2_SITE_P_READY, it)) {
         ok = false;
         break;
@@ -402,13 +436,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // B MN-major (16 query rows = 2 KiB per step)
 #pragma unroll
         for (int kk = 0; kk < kBlockM / 16; ++kk) {
-          umma_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8, bOm, idTS, (it > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + C::kColDV, tmem + C::kColS + bf16_col(kk >> 1) + 8 * (kk & 1), bOm, idTS,
+                  (it > 0 || kk > 0) ? 1u : 0u);
           bOm += (16 * kSwizzleBytes) >> 4;
         }
         umma_commit(bar(BB_OFREE + os));
 #pragma unroll
         for (int kk = 0; kk < kBlockM / 16; ++kk) {
-          umma_ts(tmem + C::kColDK, tmem + C::kColDP + kk * 8, bQm, idTS, (it > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + C::kColDK, tmem + C::kColDP + bf16_col(kk >> 1) + 8 * (kk & 1), bQm, idTS,
+                  (it > 0 || kk > 0) ? 1u : 0u);
           bQm += (16 * kSwizzleBytes) >> 4;
         }
         umma_commit(bar(BB_QFREE + qs));
@@ -423,6 +459,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         umma_commit(bar(BB_DQ));
       }
       __syncwarp();
+      // the next tile's dP^T may start now (its columns were last read by the
+      // dK MMA above, and MMAs of one thread run in issue order)
+      if (it + 1 < n_it && !issue_s_dp(it + 1)) {
+        ok = false;
+        break;
+      }
     }
     // drain: every MMA complete before dK / dV are read and TMEM is freed
     const WaitGuard drain{0u, p.limit_ns};

@@ -243,6 +243,7 @@ enum fa2_wait_site {
   FA2_SITE_FINAL_STATS = 9,
   FA2_SITE_MMA_DRAIN = 10,
   FA2_SITE_LOAD_DRAIN = 11,
+  FA2_SITE_SMEM_ALIGN = 13,   /* backward: shared memory base too far from 1 KiB alignment; not run */
   FA2_SITE_SELFTEST = 15
 };
 

@@ -1,11 +1,15 @@
 // fa2_forward.cu -- exact attention forward pass for B200 (sm_100a).
 //
-// One CTA owns 256 query rows of one (batch, query head): two 128-row query
-// tiles, Q0 and Q1, that take turns on the tensor cores.  The grid runs over
-// (query block, head, batch) -- the sequence parallelism of "FlashAttention 2:
-// Three Places the Chip Was Still Waiting", section 2.3 -- so a single long
-// head still fills the machine.  Within the CTA, work is split by role rather
-// than by data:
+// A unit of work is 256 query rows of one (batch, query head): two 128-row
+// query tiles, Q0 and Q1, that take turns on the tensor cores.  fa2_forward
+// runs one CTA per unit over (query block, head, batch) -- the sequence
+// parallelism of "FlashAttention 2: Three Places the Chip Was Still Waiting",
+// section 2.3 -- so a single long head still fills the machine;
+// fa2_forward_ws runs persistent CTAs over equal ranges of the units' work
+// (stream-K) and merges split units in a second kernel; fa2_forward_local
+// narrows each unit to the key tiles its sliding window can see.  The backward
+// pass lives in fa2_backward.cuh, compiled into this translation unit.
+// Within the CTA, work is split by role rather than by data:
 //
 //   warps 0-3   softmax for Q0, one thread per query row (TMEM lane == row), so
 //   warps 4-7   softmax for Q1   row statistics never leave a thread (the
@@ -15,7 +19,7 @@
 //               moved, and the epilogue (the single 1/l division, section 2.2)
 //   warp 12     MMA issuer: tcgen05 S = Q K^T and O += P V into TMEM
 //   warp 13     TMA producer: Q once, then K_j / V_j through a smem ring
-//   warps 14-15 idle (they only complete the fourth warpgroup)
+//   warps 14-15 rows of units that see no key at all (O = 0, LSE = -inf)
 //
 // TMEM columns: S0 | S1 | O0 | O1 (fp32).  P (bf16) is written by the softmax
 // threads over the first half of their own S tile and consumed from TMEM by

@@ -74,11 +74,23 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+KERNEL_FILES = ("fa2_forward.cu", "fa2_backward.cuh", "sm100_ptx.cuh")
+
+
+def _code_only(text: str) -> str:
+    """C/C++ source with comments and blank lines removed (so that editing a
+    comment does not retire a profile taken on the same code)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash() -> str:
+    """Hash of the code (comments stripped) of every file compiled into the kernels."""
     h = hashlib.sha256()
-    for f in (KERNEL_SRC, os.path.join(ROOT, "exact_tiled_attention_29_b200", "csrc", "sm100_ptx.cuh")):
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+    for name in KERNEL_FILES:
+        with open(os.path.join(ROOT, "exact_tiled_attention_29_b200", "csrc", name)) as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -94,10 +94,10 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, kernel: str = "fa2_fwd_kernel"):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", f"fa2_fwd_kernel_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -558,7 +558,7 @@ def run_fa2_backward(args, w):
             "dtype": "bf16", "data": "synthetic", "config": {**workload_config(w, 1), "direction": "bwd"},
             "pct_of_peak": 100.0 * achieved / peak,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak, "traffic": profiled_traffic(w.name, "fa2_bwd_kernel"),
                          "peak_source": f"bf16_tflops (burst), {peak_src}",
                          "kernel": f"fa2_bwd_kernel<{w.d}> + prep + dq rounding (timed together)"},
             "gpu_launches": 3 * args.steps, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,

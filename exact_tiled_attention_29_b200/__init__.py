@@ -7,7 +7,7 @@ does not load the library.
 """
 
 _BINDING_NAMES = {
-    "fa2_forward", "fa2_forward_local", "fa2_forward_ws", "fa2_backward",
+    "fa2_forward", "fa2_forward_local", "fa2_forward_ws", "fa2_backward", "fa2_backward_local",
     "fa2_backward_workspace_size", "attention_backward", "fa2_forward_static_ws", "fa2_workspace_size",
     "fa2_streamk_plan", "FA2_STATIC_WS_BYTES",
     "alloc_workspace", "fa2_status_string", "fa2_debug_status", "fa2_selftest_timeout",

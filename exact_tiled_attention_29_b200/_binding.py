@@ -51,6 +51,8 @@ def _load() -> ctypes.CDLL:
     lib.fa2_forward_static_ws.restype = ci
     lib.fa2_backward.argtypes = [vp] * 9 + [ci] * 7 + [cf, vp, cll, vp]
     lib.fa2_backward.restype = ci
+    lib.fa2_backward_local.argtypes = [vp] * 9 + [ci] * 8 + [cf, vp, cll, vp]
+    lib.fa2_backward_local.restype = ci
     lib.fa2_backward_workspace_size.argtypes = [ci] * 4
     lib.fa2_backward_workspace_size.restype = cll
     lib.fa2_workspace_size.argtypes = [ci] * 7
@@ -134,6 +136,16 @@ def fa2_backward(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causa
                                  _ptr(dk), _ptr(dv), int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
                                  int(bool(causal)), float(softmax_scale), _ptr(workspace),
                                  int(workspace_bytes), _stream(stream)))
+
+
+def fa2_backward_local(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, window_left,
+                       window_right, softmax_scale, workspace, workspace_bytes, stream) -> int:
+    """Gradients of fa2_forward_local (same window).  Returns the status."""
+    return int(_lib.fa2_backward_local(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                       _ptr(dq), _ptr(dk), _ptr(dv), int(B), int(Hq), int(Hkv),
+                                       int(Nq), int(Nk), int(d), int(window_left), int(window_right),
+                                       float(softmax_scale), _ptr(workspace), int(workspace_bytes),
+                                       _stream(stream)))
 
 
 def fa2_backward_workspace_size(B, Hq, Nq, d) -> int:
@@ -240,7 +252,7 @@ def attention(q, k, v, causal: bool = False, softmax_scale: float | None = None,
 
 
 def attention_backward(q, k, v, o, lse, dout, causal: bool = False,
-                       softmax_scale: float | None = None, stream=None, workspace=None):
+                       softmax_scale: float | None = None, stream=None, workspace=None, window=None):
     """dq, dk, dv for bf16 CUDA tensors (layouts as ``attention``) given the
     forward's o and lse and the upstream gradient dout; one call to
     ``fa2_backward``.  ``workspace`` (uint8 CUDA tensor of at least
@@ -257,8 +269,16 @@ def attention_backward(q, k, v, o, lse, dout, causal: bool = False,
         workspace = torch.empty(fa2_backward_workspace_size(B, Hq, Nq, d), dtype=torch.uint8,
                                 device=q.device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    st = fa2_backward(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal,
-                      softmax_scale, workspace, workspace.numel() * workspace.element_size(), stream)
+    nbytes = workspace.numel() * workspace.element_size()
+    if window is not None:
+        wl, wr = int(window[0]), int(window[1])
+        if causal:
+            wr = 0
+        st = fa2_backward_local(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, wl, wr,
+                                softmax_scale, workspace, nbytes, stream)
+    else:
+        st = fa2_backward(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal,
+                          softmax_scale, workspace, nbytes, stream)
     if st != FA2_OK:
         raise FA2Error(st, "fa2_backward")
     return dq, dk, dv

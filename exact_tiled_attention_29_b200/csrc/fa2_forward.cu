@@ -1435,10 +1435,10 @@ extern "C" long long fa2_backward_workspace_size(int B, int Hq, int Nq, int d) {
   return bwd_workspace_bytes(B, Hq, Nq, d);
 }
 
-extern "C" int fa2_backward(const void* q, const void* k, const void* v, const void* o,
-                            const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
-                            int Hq, int Hkv, int Nq, int Nk, int d, int causal, float softmax_scale,
-                            void* workspace, long long workspace_bytes, void* stream) {
+static int backward_impl(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                         int Hq, int Hkv, int Nq, int Nk, int d, Window win, float softmax_scale,
+                         void* workspace, long long workspace_bytes, void* stream) {
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
     return FA2_ERR_NULL_POINTER;
   const int sv = validate_shape(B, Hq, Hkv, Nq, Nk, d);
@@ -1456,10 +1456,30 @@ extern "C" int fa2_backward(const void* q, const void* k, const void* v, const v
   if (dv_ != FA2_OK) return dv_;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 128)
-    return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, causal_window(causal),
-                           softmax_scale, workspace, s);
-  return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, causal_window(causal),
-                        softmax_scale, workspace, s);
+    return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, win, softmax_scale,
+                           workspace, s);
+  return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, win, softmax_scale,
+                        workspace, s);
+}
+
+extern "C" int fa2_backward(const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                            int Hq, int Hkv, int Nq, int Nk, int d, int causal, float softmax_scale,
+                            void* workspace, long long workspace_bytes, void* stream) {
+  return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, causal_window(causal),
+                       softmax_scale, workspace, workspace_bytes, stream);
+}
+
+extern "C" int fa2_backward_local(const void* q, const void* k, const void* v, const void* o,
+                                  const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                  int B, int Hq, int Hkv, int Nq, int Nk, int d, int window_left,
+                                  int window_right, float softmax_scale, void* workspace,
+                                  long long workspace_bytes, void* stream) {
+  if (window_left < -1 || window_right < -1) return FA2_ERR_WINDOW;
+  // widths reaching past every key are no bound (as in fa2_forward_local)
+  const Window w{window_left >= Nk ? -1 : window_left, window_right >= Nq ? -1 : window_right};
+  return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, w, softmax_scale,
+                       workspace, workspace_bytes, stream);
 }
 
 extern "C" long long fa2_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal) {

@@ -216,6 +216,19 @@ int fa2_backward(const void* q, const void* k, const void* v, const void* o, con
                  int Nk, int d, int causal, float softmax_scale, void* workspace,
                  long long workspace_bytes, void* stream);
 
+/*
+ * fa2_backward_local -- fa2_backward for fa2_forward_local's window: key j is
+ * visible to row i when g - window_left <= j <= g + window_right,
+ * g = i + Nk - Nq (-1 leaves a side open).  o and lse must come from
+ * fa2_forward_local with the same window.  FA2_ERR_WINDOW for a width below
+ * -1; otherwise as fa2_backward.
+ */
+int fa2_backward_local(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
+                       int Nq, int Nk, int d, int window_left, int window_right,
+                       float softmax_scale, void* workspace, long long workspace_bytes,
+                       void* stream);
+
 /* Bytes of scratch fa2_backward needs (-1 for invalid arguments). */
 long long fa2_backward_workspace_size(int B, int Hq, int Nq, int d);
 

@@ -4,7 +4,9 @@ Tolerance, derived from the arithmetic: P and dS enter the tensor cores as
 bf16 (relative rounding 2^-9), are accumulated in fp32, and dS also carries
 the forward's bf16 O through D = dO . O.  Each gradient is compared relative
 to its own scale: max |err| <= 3e-2 * max |ref| and mean |err| <= 1e-2 *
-mean |ref|, with no NaN or Inf.
+mean |ref|, with no NaN or Inf.  Where a gradient vanishes exactly (a row that
+sees one key has dS = P (dP - D) = 0) the GPU's dP - D is a rounding residue,
+so the scales have floors: 1e-3 for the max and 1e-4 for the mean.
 """
 
 import numpy as np
@@ -46,9 +48,9 @@ def check(fa2, w, scale=None):
     for name, a, r in zip(("dQ", "dK", "dV"), got, ref):
         assert np.isfinite(a).all(), f"{w.name}: non-finite {name}"
         err = np.abs(a - r)
-        big = max(np.abs(r).max(), 1e-6)
+        big = max(np.abs(r).max(), 1e-3)
         assert err.max() <= MAX_REL * big, f"{w.name} {name}: max err {err.max():.3g} vs scale {big:.3g}"
-        assert err.mean() <= MEAN_REL * max(np.abs(r).mean(), 1e-9), \
+        assert err.mean() <= MEAN_REL * max(np.abs(r).mean(), 1e-4), \
             f"{w.name} {name}: mean err {err.mean():.3g} vs mean {np.abs(r).mean():.3g}"
 
 
@@ -72,3 +74,26 @@ def test_backward_deterministic_dk_dv(fa2):
     a = grads_gpu(fa2, q, k, v, g, True, w.softmax_scale)
     b = grads_gpu(fa2, q, k, v, g, True, w.softmax_scale)
     assert np.array_equal(a[1], b[1]) and np.array_equal(a[2], b[2])
+
+
+@pytest.mark.parametrize("window", [(0, 0), (127, 0), (300, -1), (200, 100), (-1, 50)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_local_window(fa2, window, d):
+    w = Workload("bwd_loc", 2, 4, 2, 700, 650, d, False, seed=60 + d)
+    q, k, v = make_qkv(w)
+    g = torch.randn(q.shape, generator=torch.Generator().manual_seed(61)).to(torch.bfloat16)
+    dev = torch.device("cuda")
+    qd, kd, vd, gd = (t.to(dev) for t in (q, k, v, g))
+    o, lse = fa2.attention(qd, kd, vd, window=window)
+    got = [t.float().cpu().numpy()
+           for t in fa2.attention_backward(qd, kd, vd, o, lse, gd, window=window)]
+    torch.cuda.synchronize()
+    assert fa2.fa2_debug_status(None) == 0
+    ref = oracle.backward(bf16_bits(q), bf16_bits(k), bf16_bits(v), bf16_bits(g), False,
+                          w.softmax_scale, window=window)
+    for name, a, r in zip(("dQ", "dK", "dV"), got, ref):
+        assert np.isfinite(a).all(), f"{window} non-finite {name}"
+        err = np.abs(a - r)
+        big = max(np.abs(r).max(), 1e-3)
+        assert err.max() <= MAX_REL * big, f"{window} {name}: max err {err.max():.3g} vs {big:.3g}"
+        assert err.mean() <= MEAN_REL * max(np.abs(r).mean(), 1e-4), f"{window} {name}: mean err"

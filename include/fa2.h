@@ -52,7 +52,10 @@ enum fa2_status_code {
 };
 
 /*
- * fa2_forward -- enqueue one attention forward pass on `stream`.
+ * fa2_forward -- enqueue one attention forward pass on `stream` (one kernel:
+ * a block per unit of 256 query rows, or, with at least two units per SM,
+ * one persistent block per SM that takes whole units round robin so the next
+ * unit's loads overlap the current one's drain; same arithmetic either way).
  *
  *   q    device pointer, bf16 [B, Nq, Hq,  d], contiguous (d fastest); read only
  *   k    device pointer, bf16 [B, Nk, Hkv, d], contiguous; read only
@@ -277,8 +280,11 @@ int fa2_selftest_timeout(void* stream, long long limit_ns);
  * "FlashAttention 2: Three Places the Chip Was Still Waiting", section 2.3.
  * Returns -1 on non-positive arguments.
  *
- * fa2_launch_plan: the launch this library uses for a problem: grid size,
- * threads per block, dynamic shared memory bytes and query rows per block.
+ * fa2_launch_plan: the work decomposition fa2_forward uses for a problem:
+ * the number of units (256 query rows of one head and batch each, one thread
+ * block apiece when there are fewer than two units per SM; otherwise one
+ * persistent block per SM takes whole units round robin, heaviest first),
+ * threads per block, dynamic shared memory bytes and query rows per unit.
  * Returns an fa2_status_code (validation as in fa2_forward, minus pointers).
  */
 long long fa2_num_blocks(int B, int H, int N, int rows_per_block);

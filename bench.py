@@ -319,6 +319,11 @@ def run_fa2(args, w):
     # is split, the combine kernel.
     ws = None
     launches_per_step = 1
+    # the library runs whole units on persistent CTAs when there are at least
+    # two units per SM (the persistent instantiation of the kernel)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    persistent = args.schedule == "streamk" or fa2.fa2_launch_plan(
+        w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d)[1] >= 2 * sms
     if args.schedule == "streamk" and w.windowed:
         raise SystemExit("the local-window workloads run the one-block-per-unit schedule only")
     if args.schedule == "streamk":
@@ -443,7 +448,7 @@ def run_fa2(args, w):
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"bf16_tflops (burst, kernel timed alone), {peak_src}",
                          "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"]),
-                         "kernel": f"fa2_fwd_kernel<{w.d}, {'true' if ws is not None else 'false'}>"
+                         "kernel": f"fa2_fwd_kernel<{w.d}, {'true' if persistent else 'false'}>"
                                    + (" + fa2_combine_kernel (timed together)" if launches_per_step > 1 else "")},
             "hbm_gbs_compulsory": w.compulsory_bytes() / (mean_ms * 1e-3) / 1e9,
             "bracket_ms_per_step_incl_flush": bracket_ms / args.steps,

@@ -227,7 +227,7 @@ struct Piece {
   int nt0, nt1;     // K/V tiles of Q0 / Q1 over the whole unit
   int a0, a1;       // iterations of Q0 / Q1 in this piece
   int split;        // the unit is shared with other pieces
-  int slot;         // CTA that runs the unit's first piece (its counter is the unit's)
+  int slot;         // CTA that runs the unit's first piece (the partial buffers count from it)
   int npieces;      // pieces of the unit
   int index;        // this piece's position in the unit
 };
@@ -353,7 +353,7 @@ struct PieceIter {
       r = u / HB;
       k_cur = u % HB;
       const int nn = unit_tiles(p.Nq, p.Nk, window_of(p), p.n_qblk - 1 - r);
-      if (nn == 0) return false;  // nothing to compute: the merge warps write this unit's empty rows
+      if (nn == 0) return false;  // nothing to compute: warps 14-15 write this unit's empty rows
       cum = 0;
       n = nn;
       fill(p, pc, r, k_cur, 0, nn);

@@ -183,3 +183,28 @@ def test_forward_ws_validation(over, code):
 def test_workspace_size_rejects_bad_shapes():
     assert fa2.fa2_workspace_size(0, 1, 1, 1, 1, 128, 0) == -1
     assert fa2.fa2_workspace_size(1, 3, 2, 1, 1, 128, 0) == -1
+
+
+def persistent_units_of_cta(c, G, U):
+    """Units CTA c takes when whole units are dealt round robin, alternating
+    direction each wave (the kernel's persistent-units schedule)."""
+    out, w = [], 0
+    while True:
+        u = w * G + ((G - 1 - c) if (w & 1) else c)
+        if u >= U:
+            return out
+        out.append(u)
+        w += 1
+
+
+@pytest.mark.parametrize("B,Hq,Nq,causal,G", [(2, 16, 8192, 1, 148), (4, 16, 2048, 0, 148),
+                                              (4, 32, 4096, 1, 148), (1, 3, 5000, 1, 7)])
+def test_persistent_units_deal_every_unit_once_and_pair_heavy_with_light(B, Hq, Nq, causal, G):
+    units = list(units_in_order(B, Hq, Nq, Nq, causal))
+    U = len(units)
+    dealt = [persistent_units_of_cta(c, G, U) for c in range(G)]
+    flat = sorted(u for d in dealt for u in d)
+    assert flat == list(range(U))
+    loads = [sum(units[u][2] for u in d) for d in dealt]
+    # a CTA's load differs from the mean by less than one unit of the heaviest size
+    assert max(loads) - min(loads) <= max(n for _, _, n in units)

@@ -253,3 +253,17 @@ def test_small_workspace_is_refused(fa2):
     st = fa2.fa2_forward_ws(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
                             w.softmax_scale, ws, ws.numel(), torch.cuda.current_stream())
     assert st == 10
+
+
+# ---- the persistent whole-unit schedule fa2_forward takes with >= 2 units per SM ----
+
+@pytest.mark.parametrize("w", [
+    Workload("pu_d64", 4, 16, 16, 2048, 2048, 64, False, seed=71),          # 512 units, d = 64
+    Workload("pu_nq_gt_nk", 8, 8, 4, 3000, 1500, 64, True, seed=72),        # 768 units, leading ones empty
+    Workload("pu_gqa_ragged", 3, 24, 6, 1900, 1900, 128, True, seed=73),    # 576 units, ragged tail
+])
+def test_persistent_units_schedule(fa2, w):
+    st, units, _, _, _ = fa2.fa2_launch_plan(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d)
+    assert st == 0 and units >= 2 * torch.cuda.get_device_properties(0).multi_processor_count
+    rows = sample_rows(w, 300, seed=74)
+    check_case(fa2, w, rows=rows)

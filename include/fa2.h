@@ -1,7 +1,8 @@
 /*
- * fa2.h -- C ABI of the B200 (sm_100a) exact attention forward pass.
+ * fa2.h -- C ABI of the B200 (sm_100a) exact attention forward and backward
+ * passes.
  *
- * The library computes, for every batch b, query head hq and query row i,
+ * The forward computes, for every batch b, query head hq and query row i,
  *
  *     O[b,i,hq,:] = softmax_j( softmax_scale * q[b,i,hq,:] . k[b,j,hk,:] ) v[b,j,hk,:]
  *     LSE[b,hq,i] = ln sum_j exp( softmax_scale * q[b,i,hq,:] . k[b,j,hk,:] )
@@ -24,9 +25,11 @@
  *   - a row with no visible key gets O = 0 and LSE = -inf;
  *   - LSE is the natural log and includes softmax_scale.
  *
- * All entry points are thread-safe and allocate no device memory; the
- * stream-K variant takes its scratch memory from the caller, or from a fixed
- * array of the library (fa2_forward_static_ws, whose calls must not overlap).
+ * and the backward (fa2_backward) its gradients.  All entry points are
+ * thread-safe and allocate no device memory; the stream-K forward and the
+ * backward take their scratch memory from the caller, or (stream-K only) from
+ * a fixed array of the library (fa2_forward_static_ws, whose calls must not
+ * overlap).
  */
 #ifndef FA2_H
 #define FA2_H

@@ -31,6 +31,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -1204,32 +1205,41 @@ static int sm_count() {
   return n;
 }
 
+// Devices the per-device set-up below can track (device ordinals 0 .. 63).
+constexpr int kMaxDevices = 64;
+
+// Runs `setup` once per device (the current one) and returns its status on
+// every later call.  Function attributes such as the dynamic shared-memory
+// limit are per device, so a process that calls the library on several GPUs
+// sets them up on each.
+template <typename F>
+static int once_per_device(std::once_flag (&flags)[kMaxDevices], int (&status)[kMaxDevices], F setup) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA2_ERR_DEVICE;
+  std::call_once(flags[dev], [&] { status[dev] = setup(); });
+  return status[dev];
+}
+
 template <int D>
 static int launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                   int Hkv, int Nq, int Nk, Window win, float scale, void* workspace,
                   long long workspace_bytes, cudaStream_t stream, bool persistent_units) {
   using C = Cfg<D>;
-  static std::once_flag once;
-  static int setup_status = FA2_OK;
-  std::call_once(once, [] {
+  static std::once_flag flags[kMaxDevices];
+  static int setup_status[kMaxDevices];
+  const int st = once_per_device(flags, setup_status, [] {
     for (auto* kern : {fa2_fwd_kernel<D, false>, fa2_fwd_kernel<D, true>}) {
       cudaFuncAttributes attr;
-      if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) {
-        setup_status = FA2_ERR_LAUNCH;
-        return;
-      }
-      if (attr.numRegs != kLaunchRegs) {  // the setmaxnreg split assumes exactly this pool
-        setup_status = FA2_ERR_BUILD;
-        return;
-      }
+      if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return static_cast<int>(FA2_ERR_LAUNCH);
+      // the setmaxnreg split assumes exactly this pool
+      if (attr.numRegs != kLaunchRegs) return static_cast<int>(FA2_ERR_BUILD);
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
-          cudaSuccess) {
-        setup_status = FA2_ERR_LAUNCH;
-        return;
-      }
+          cudaSuccess)
+        return static_cast<int>(FA2_ERR_LAUNCH);
     }
+    return static_cast<int>(FA2_OK);
   });
-  if (setup_status != FA2_OK) return setup_status;
+  if (st != FA2_OK) return st;
 
   Params p;
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -1306,14 +1316,15 @@ static int launch_bwd(const void* q, const void* k, const void* v, const void* o
                       const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
                       int Nk, Window win, float scale, void* workspace, cudaStream_t stream) {
   using C = BCfg<D>;
-  static std::once_flag once;
-  static int setup_status = FA2_OK;
-  std::call_once(once, [] {
-    if (cudaFuncSetAttribute(fa2_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
-      setup_status = FA2_ERR_LAUNCH;
+  static std::once_flag flags[kMaxDevices];
+  static int setup_status[kMaxDevices];
+  const int st = once_per_device(flags, setup_status, [] {
+    return cudaFuncSetAttribute(fa2_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                C::kSmemBytes) == cudaSuccess
+               ? static_cast<int>(FA2_OK)
+               : static_cast<int>(FA2_ERR_LAUNCH);
   });
-  if (setup_status != FA2_OK) return setup_status;
+  if (st != FA2_OK) return st;
   const long long rows = static_cast<long long>(B) * Nq * Hq;
   float* dq_acc = static_cast<float*>(workspace);
   float* lse2 = dq_acc + ((rows * D + 63) / 64) * 64;
@@ -1359,36 +1370,43 @@ static long long bwd_workspace_bytes(int B, int Hq, int Nq, int d) {
 }
 
 static int check_device() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return FA2_ERR_DEVICE;
-  static int cached[64];
-  static std::once_flag flags[64];
-  if (dev < 0 || dev >= 64) return FA2_ERR_DEVICE;
-  std::call_once(flags[dev], [dev] {
-    int major = 0, minor = 0;
-    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-    cached[dev] = (major == 10 && minor == 0) ? FA2_OK : FA2_ERR_DEVICE;
+  static std::once_flag flags[kMaxDevices];
+  static int cached[kMaxDevices];
+  return once_per_device(flags, cached, [] {
+    int dev = 0, major = 0, minor = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return static_cast<int>(FA2_ERR_DEVICE);
+    return (major == 10 && minor == 0) ? static_cast<int>(FA2_OK) : static_cast<int>(FA2_ERR_DEVICE);
   });
-  return cached[dev];
 }
 
 }  // namespace fa2
 
 using namespace fa2;
 
-static int forward_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                        int Hq, int Hkv, int Nq, int Nk, int d, Window win, float softmax_scale,
-                        void* workspace, long long workspace_bytes, void* stream) {
+// The checks of the forward entry points that need no CUDA call: pointers,
+// shape, alignment (TMA needs 16-byte aligned q, k, v, o), the scale.
+static int validate_args(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         int B, int Hq, int Hkv, int Nq, int Nk, int d, float softmax_scale) {
   if (!q || !k || !v || !o || !lse) return FA2_ERR_NULL_POINTER;
   const int sv = validate_shape(B, Hq, Hkv, Nq, Nk, d);
   if (sv != FA2_OK) return sv;
   if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
-       reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o) |
-       reinterpret_cast<uintptr_t>(workspace)) & 15u)
+       reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o)) & 15u)
     return FA2_ERR_ALIGNMENT;
   if (reinterpret_cast<uintptr_t>(lse) & 3u) return FA2_ERR_ALIGNMENT;
   if (!std::isfinite(softmax_scale)) return FA2_ERR_SCALE;
+  return FA2_OK;
+}
+
+static int forward_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int Nq, int Nk, int d, Window win, float softmax_scale,
+                        void* workspace, long long workspace_bytes, void* stream) {
+  const int sa = validate_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, softmax_scale);
+  if (sa != FA2_OK) return sa;
+  if (reinterpret_cast<uintptr_t>(workspace) & 15u) return FA2_ERR_ALIGNMENT;
   if (workspace && workspace_bytes < 0) return FA2_ERR_WORKSPACE;
   const int dv = check_device();
   if (dv != FA2_OK) return dv;
@@ -1441,30 +1459,32 @@ extern "C" int fa2_forward_ws(const void* q, const void* k, const void* v, void*
 constexpr size_t kStaticScratchBytes = FA2_STATIC_WS_BYTES;  // 2 partials x 148 SMs at d = 128 fit
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-// Device address of the array on device `dev` (the current device), looked
-// up once per device and cached; nullptr if the lookup failed.
+// Device address of the array on device `dev` (the current device), or
+// nullptr if it cannot be obtained.  Only a successful lookup is kept: a
+// failed one (for instance made while the stream was being captured) is
+// retried by the next call.
 static void* static_scratch(int dev) {
-  static void* addr[64];
-  static std::once_flag flags[64];
-  std::call_once(flags[dev], [dev] {
-    void* a = nullptr;
-    if (cudaGetSymbolAddress(&a, g_static_scratch) == cudaSuccess) addr[dev] = a;
-  });
-  return addr[dev];
+  static std::atomic<void*> addr[kMaxDevices];
+  void* a = addr[dev].load(std::memory_order_acquire);
+  if (a) return a;
+  if (cudaGetSymbolAddress(&a, g_static_scratch) != cudaSuccess || !a) {
+    cudaGetLastError();  // clear it, so a later launch check does not report it
+    return nullptr;
+  }
+  addr[dev].store(a, std::memory_order_release);  // the same value whichever thread stores it
+  return a;
 }
 
 extern "C" int fa2_forward_static_ws(const void* q, const void* k, const void* v, void* o, float* lse,
                                      int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
                                      float softmax_scale, void* stream) {
-  // the checks fa2_forward makes before touching CUDA, then the device
-  if (!q || !k || !v || !o || !lse) return FA2_ERR_NULL_POINTER;
-  const int sv = validate_shape(B, Hq, Hkv, Nq, Nk, d);
+  // every argument check fa2_forward makes, in its order, before any CUDA call
+  const int sv = validate_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, softmax_scale);
   if (sv != FA2_OK) return sv;
-  if (!std::isfinite(softmax_scale)) return FA2_ERR_SCALE;
   const int dv = check_device();
   if (dv != FA2_OK) return dv;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FA2_ERR_DEVICE;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA2_ERR_DEVICE;
   void* scratch = static_scratch(dev);
   if (!scratch) return FA2_ERR_LAUNCH;
   // a problem whose plan needs more than the array is refused (FA2_ERR_WORKSPACE)

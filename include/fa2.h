@@ -180,7 +180,10 @@ long long fa2_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int 
  *
  * The array's address is looked up once per device (cudaGetSymbolAddress,
  * with that device current) on the first call on that device; make that first
- * call before capturing the stream into a CUDA graph.  All calls on a device
+ * call before capturing the stream into a CUDA graph.  A lookup that fails is
+ * not remembered: the call returns FA2_ERR_LAUNCH and the next call tries
+ * again.  Argument checks (pointers, shape, alignment, scale) come before any
+ * CUDA call, as in fa2_forward.  All calls on a device
  * share the one array: calls that may overlap in time (unordered streams,
  * several host threads) race on it and give wrong results -- order them on
  * one stream.

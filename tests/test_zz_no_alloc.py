@@ -32,6 +32,10 @@ def test_static_validation_before_any_cuda_call():
     assert fa2.fa2_forward_static_ws(16, 32, 48, 64, 80, 1, 3, 2, 5, 7, 128, 1, 0.1, None) == 2
     assert fa2.fa2_forward_static_ws(16, 32, 48, 64, 80, 1, 2, 1, 5, 7, 96, 1, 0.1, None) == 3
     assert fa2.fa2_forward_static_ws(16, 32, 48, 64, 80, 1, 2, 1, 5, 7, 128, 1, math.nan, None) == 5
+    # misaligned q / o (16 bytes) or lse (4 bytes): refused before the device is touched
+    assert fa2.fa2_forward_static_ws(24, 32, 48, 64, 80, 1, 2, 1, 5, 7, 128, 1, 0.1, None) == 4
+    assert fa2.fa2_forward_static_ws(16, 32, 48, 72, 80, 1, 2, 1, 5, 7, 128, 1, 0.1, None) == 4
+    assert fa2.fa2_forward_static_ws(16, 32, 48, 64, 82, 1, 2, 1, 5, 7, 128, 1, 0.1, None) == 4
     if not torch.cuda.is_available():
         assert call_static(args["q"], args["k"], args["v"], args["o"], args["lse"], w) == 6
 

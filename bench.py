@@ -8,8 +8,9 @@ synthetic inputs, already resident in HBM.  L2 is flushed (a 256 MiB write)
 before every step, outside the per-step CUDA events that time the launch on
 its own stream.  ``value`` = algorithmic TFLOP/s of all ranks (4*B*Hq*Nq*Nk*d,
 halved when causal) / max-over-ranks mean step time.  With N > 1 (torchrun),
-each rank runs its own independently seeded batch of the same workload (weak
-scaling; the ranks exchange nothing but the timing reduction).
+the job is one problem whose KV-head groups are split over the ranks, each
+rank holding one workload's worth of heads (weak scaling; the ranks exchange
+nothing but the timing reduction).
 
 ``e2e`` measures the same metric through the public API with host buffers:
 pinned-host Q/K/V -> device, the C-ABI call, O and LSE -> pinned host.
@@ -35,7 +36,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from exact_tiled_attention_29_b200.inputs import (EXTRA_WORKLOADS, WORKLOADS, bf16_bits,  # noqa: E402
-                                                  make_qkv)
+                                                  make_qkv, shard_seed)
 
 ALL_WORKLOADS = {**WORKLOADS, **EXTRA_WORKLOADS}
 
@@ -278,9 +279,10 @@ def run_reference(args, w):
 
 
 def rank_seed(w, rank: int) -> int:
-    """Seed of rank `rank`'s independent batch (weak scaling: every rank runs
-    the full workload on its own inputs)."""
-    return w.seed + rank
+    """Seed of rank `rank`'s share of the job: its KV-head groups of the whole
+    problem (``inputs.global_workload``), drawn independently of the other
+    ranks' (weak scaling: every rank holds one workload's worth of heads)."""
+    return shard_seed(w, rank)
 
 
 def max_over_ranks(values, device=None):
@@ -308,7 +310,9 @@ def workload_config(w, n_gpus, schedule="units"):
     return {**cfg,
             "softmax_scale": w.softmax_scale, "seed": w.seed,
             "flops_per_step_per_rank": w.flops(),
-            "parallelism": f"independent batches per rank x{n_gpus}" if n_gpus > 1 else "single GPU",
+            "parallelism": (f"KV-head groups split over {n_gpus} ranks (rank r: query heads "
+                            f"[r*{w.Hq}, (r+1)*{w.Hq}), KV heads [r*{w.Hkv}, (r+1)*{w.Hkv})), "
+                            "no collective on the data path") if n_gpus > 1 else "single GPU",
             "l2": "flushed before every step (256 MiB write), outside the per-step events"}
 
 

@@ -131,6 +131,27 @@ def make_qkv(w: Workload, seed: int | None = None):
     return (q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16))
 
 
+def shard_seed(w: Workload, rank: int) -> int:
+    """Seed of rank `rank`'s share of a multi-GPU job (rank 0's equals the
+    single-GPU inputs)."""
+    return w.seed + rank
+
+
+def global_workload(w: Workload, world: int) -> Workload:
+    """The whole job of `world` ranks that each hold workload `w`: the KV-head
+    groups of one problem are split across the ranks, rank r holding query
+    heads [r*Hq, (r+1)*Hq) and KV heads [r*Hkv, (r+1)*Hkv) (whole groups, so
+    no rank needs another's K or V)."""
+    return w.with_(name=f"{w.name}_x{world}", Hq=w.Hq * world, Hkv=w.Hkv * world)
+
+
+def make_global_qkv(w: Workload, world: int):
+    """Inputs of the whole job in the single-GPU layout ``[B, N, H, d]``: rank
+    r's head slice is ``make_qkv(w, seed=shard_seed(w, r))``."""
+    parts = [make_qkv(w, seed=shard_seed(w, r)) for r in range(world)]
+    return tuple(torch.cat([p[i] for p in parts], dim=2) for i in range(3))
+
+
 def sample_rows(w: Workload, n_sample: int = 1024, seed: int | None = None) -> np.ndarray:
     """Seeded sample of query rows used when every row is too many for the oracle.
 

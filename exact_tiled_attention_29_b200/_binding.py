@@ -71,6 +71,8 @@ def _load() -> ctypes.CDLL:
     llp = ctypes.POINTER(cll)
     lib.fa2_streamk_plan.argtypes = [ci] * 8 + [llp, ip, llp]
     lib.fa2_streamk_plan.restype = ci
+    lib.fa2_persistent_plan.argtypes = [ci] * 8 + [ip, ip, ci]
+    lib.fa2_persistent_plan.restype = ci
     return lib
 
 
@@ -164,6 +166,19 @@ def fa2_streamk_plan(B, Hq, Hkv, Nq, Nk, d, causal, num_sms):
                                int(bool(causal)), int(num_sms), ctypes.byref(t), ctypes.byref(g),
                                ctypes.byref(w))
     return int(st), t.value, g.value, w.value
+
+
+def fa2_persistent_plan(B, Hq, Hkv, Nq, Nk, d, causal, num_sms, capacity=1 << 14):
+    """(status, start, units): block c of the persistent launch runs
+    units[start[c]:start[c + 1]] in that order."""
+    start = (ctypes.c_int * (num_sms + 1))()
+    units = (ctypes.c_int * capacity)()
+    st = _lib.fa2_persistent_plan(int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
+                                  int(bool(causal)), int(num_sms), start, units, int(capacity))
+    if st != 0:
+        return int(st), [], []
+    n = start[num_sms]
+    return 0, list(start), list(units[:n])
 
 
 def fa2_status_string(status: int) -> str:

@@ -15,15 +15,16 @@
 //   warps 4-7   softmax for Q1   row statistics never leave a thread (the
 //                                "partition on the index that survives to the
 //                                output" rule, section 2.4)
-//   warps 8-11  correction: rescales the O accumulator in TMEM when a row max
-//               moved, and the epilogue (the single 1/l division, section 2.2)
+//   warps 8-11  correction: rescales the O accumulator in TMEM when a row's
+//               reference max is raised, and the epilogue (the single 1/l
+//               division, section 2.2)
 //   warp 12     MMA issuer: tcgen05 S = Q K^T and O += P V into TMEM
 //   warp 13     TMA producer: Q once, then K_j / V_j through a smem ring
 //   warps 14-15 rows of units that see no key at all (O = 0, LSE = -inf)
 //
 // TMEM columns: S0 | S1 | O0 | O1 (fp32).  P (bf16) is written by the softmax
-// threads over the first half of their own S tile and consumed from TMEM by
-// the PV MMA.  The overlap of loads, matrix products and softmax follows the
+// threads over the first half of its own S tile and consumed from TMEM by
+// the PV MMA, in two halves of 64 keys, each as soon as it is written.  The overlap of loads, matrix products and softmax follows the
 // producer/consumer idea of "FlashAttention-2 and -3: From Algebra to GPU
 // Scheduling", "FlashAttention-3: overlap work on Hopper", rebuilt for
 // tcgen05/TMEM.
@@ -32,12 +33,16 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <queue>
 #include <type_traits>
+#include <utility>
+#include <vector>
 
 #include "../../include/fa2.h"
 #include "sm100_ptx.cuh"
@@ -67,13 +72,14 @@ enum Bar {
   BAR_Q = 0,         // Q tiles of the current piece loaded (TMA tx)
   BAR_QFREE = 1,     // the current piece's last S MMA completed: Q smem reusable (MMA commit)
   BAR_S = 2,         // [2] S tile complete (MMA commit)
-  BAR_P = 4,         // [2] P written to TMEM and O rescaled (128 softmax + 128 correction threads)
+  BAR_P = 4,         // [2] keys 64-127 of P written to TMEM (128 softmax threads)
   BAR_STATS = 6,     // [2] per-row rescale factor published (128 softmax threads)
   BAR_OFINAL = 8,    // [2] last PV of a piece complete (MMA commit)
   BAR_FSTATS = 10,   // [2] final row max / denominator of a piece published (128 softmax threads)
   BAR_FCONS = 12,    // [2] final statistics read by the epilogue (128 correction threads)
   BAR_DONE = 14,     // all MMAs drained (MMA commit)
-  BAR_KV_FULL = 15,  // [stages] K/V tile landed (TMA tx); then [stages] slot free (MMA commit)
+  BAR_PH = 15,       // [2] keys 0-63 of P written and O rescaled (128 softmax + 128 correction threads)
+  BAR_KV_FULL = 17,  // [stages] K/V tile landed (TMA tx); then [stages] slot free (MMA commit)
 };
 
 // Scheduling cost of a unit, in K/V-tile iterations, on top of its
@@ -93,6 +99,29 @@ constexpr int kUnitCost = 2;
 #endif
 constexpr bool kPersistentUnits = FA2_PERSISTENT_UNITS != 0;
 
+// Lazy rescaling: a row's exponentials and its O accumulator are taken
+// relative to a reference max that is raised to the running max only when the
+// running max exceeds it by more than this many log2 units (a factor of 256).
+// O and the denominator l always share the reference, so the result is the
+// same in exact arithmetic; every probability stays <= 2^8 and l <= 2^8 Nk,
+// far inside fp32.  On random data the reference settles after the first tile
+// and O is almost never touched again ("FlashAttention 2: Three Places the Chip
+// Was Still Waiting", section 2.2: the correction factor is what remains in
+// the loop once the division has moved out of it).
+constexpr float kRescaleThreshold = 8.f;
+
+// Persistent whole units: the host plans which CTA runs which unit and in
+// what order, and passes the plan as a kernel parameter (no device memory).
+// Up to kMaxTableUnits units on up to kMaxTableCtas CTAs; larger problems
+// deal units round robin instead.
+constexpr int kMaxTableCtas = 160;
+constexpr int kMaxTableUnits = 8192;
+struct UnitTable {
+  uint16_t start[kMaxTableCtas + 1];  // CTA c runs unit[start[c] .. start[c+1]) in that order
+  uint16_t unit[kMaxTableUnits];      // unit index u = round * B * Hq + (b * Hq + hq)
+};
+struct NoTable {};
+
 // Warps 14-15 (otherwise idle) write the rows of units with no visible key.
 constexpr int kEmptyThreads = 64;
 
@@ -106,8 +135,9 @@ struct Cfg {
   static constexpr int kOffAlpha = kOffKV + kStages * kTileBytes;
   static constexpr int kOffM = kOffAlpha + kTiles * kBlockM * 4;
   static constexpr int kOffL = kOffM + kTiles * kBlockM * 4;
+  static constexpr int kOffLR = kOffL + kTiles * kBlockM * 4;
   static constexpr int kNumBars = BAR_KV_FULL + 2 * kStages;
-  static constexpr int kOffBar = kOffL + kTiles * kBlockM * 4;
+  static constexpr int kOffBar = kOffLR + kTiles * kBlockM * 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kUsed = kOffMisc + 16;
   static constexpr int kSmemBytes = kUsed + 1024;  // slack for 1024-byte alignment
@@ -115,13 +145,14 @@ struct Cfg {
   __host__ __device__ static constexpr uint32_t col_s(int t) { return t ? 128u : 0u; }
   __host__ __device__ static constexpr uint32_t col_o(int t) { return 256u + (t ? D : 0); }
   // floats of one stream-K partial: O as [2 tiles][D/16 chunks][128 rows][16],
-  // then m [2][128] and l [2][128]
-  static constexpr int kPieceFloats = kTiles * kBlockM * (D + 2);
+  // then m [2][128], l [2][128] and the rounding term lr [2][128]
+  static constexpr int kPieceFloats = kTiles * kBlockM * (D + 3);
   __host__ __device__ static constexpr int part_o(int t, int ch, int row) {
     return ((t * (D / 16) + ch) * kBlockM + row) * 16;
   }
   __host__ __device__ static constexpr int part_m(int t, int row) { return kTiles * kBlockM * D + t * kBlockM + row; }
   __host__ __device__ static constexpr int part_l(int t, int row) { return part_m(t, row) + kTiles * kBlockM; }
+  __host__ __device__ static constexpr int part_lr(int t, int row) { return part_l(t, row) + kTiles * kBlockM; }
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(256 + 2 * D <= (int)kTmemCols, "TMEM budget");
 };
@@ -138,7 +169,9 @@ struct Params {
   uint32_t limit_ns;  // per bounded wait
   // work decomposition
   int streamk;        // 0: CTA i runs unit i whole; 1: CTA c runs cost positions [c*T/G, (c+1)*T/G)
-  int pu;             // with the persistent kernel: whole units dealt round robin instead (no splits)
+  int pu;             // with the persistent kernel: whole units (no splits), from the plan when tab is set,
+                      // else dealt round robin
+  int tab;            // the persistent kernel's unit plan is valid
   int T;              // summed unit costs, kUnitCost + iterations per unit (< 2^31, checked on the host)
   int span;           // T / G
   int rem;            // T % G
@@ -346,7 +379,8 @@ struct PieceIter {
     }
   }
 
-  __device__ __forceinline__ bool next(const Params& p, Piece& pc) {
+  // plan: the persistent launch's unit plan (read when p.tab is set)
+  __device__ __forceinline__ bool next(const Params& p, Piece& pc, const UnitTable* plan = nullptr) {
     if constexpr (!SK) {
       if (!state) return false;
       state = 0;
@@ -366,7 +400,14 @@ struct PieceIter {
       // when w is odd) so each CTA's heavy and light units pair up.
       const int u_count = p.r_empty * HB;  // units with some visible key
       const int c = static_cast<int>(blockIdx.x);
-      const int u = x * p.G + ((x & 1) ? p.G - 1 - c : c);
+      int u;
+      if (p.tab) {
+        const int i = plan->start[c] + x;
+        if (i >= plan->start[c + 1]) return false;
+        u = plan->unit[i];
+      } else {
+        u = x * p.G + ((x & 1) ? p.G - 1 - c : c);
+      }
       ++x;
       if (u >= u_count) return false;
       r = u / HB;
@@ -448,7 +489,8 @@ constexpr int kEmuPairs = FA2_EMU_PAIRS;
 template <int D, bool SK>
 __global__ void __launch_bounds__(kThreads, 1)
     fa2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const Params p) {
+                   const __grid_constant__ CUtensorMap tmV, const Params p,
+                   const __grid_constant__ std::conditional_t<SK, UnitTable, NoTable> plan) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -457,6 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* sm_alpha = reinterpret_cast<float*>(smem + C::kOffAlpha);
   float* sm_m = reinterpret_cast<float*>(smem + C::kOffM);
   float* sm_l = reinterpret_cast<float*>(smem + C::kOffL);
+  float* sm_lr = reinterpret_cast<float*>(smem + C::kOffLR);
   const uint32_t bar0 = sbase + C::kOffBar;
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
@@ -472,9 +515,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < BAR_KV_FULL; ++i) {
       uint32_t cnt = 1;
       if ((i >= BAR_STATS && i < BAR_STATS + 2) || (i >= BAR_FSTATS && i < BAR_FSTATS + 2) ||
-          (i >= BAR_FCONS && i < BAR_FCONS + 2))
+          (i >= BAR_FCONS && i < BAR_FCONS + 2) || (i >= BAR_P && i < BAR_P + 2))
         cnt = kBlockM;
-      if (i >= BAR_P && i < BAR_P + 2) cnt = 2 * kBlockM;
+      if (i >= BAR_PH && i < BAR_PH + 2) cnt = 2 * kBlockM;
       mbar_init(bar(i), cnt);
     }
     for (int s = 0; s < 2 * C::kStages; ++s) mbar_init(bar(BAR_KV_FULL + s), 1);
@@ -494,6 +537,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitGuard g{smem_addr(const_cast<int*>(abort_flag)), p.limit_ns};
+  const UnitTable* unit_plan = nullptr;  // the host's plan of whole units (read when p.tab is set)
+  if constexpr (SK) unit_plan = &plan;
   const bool aligned_ok = (sbase & 1023u) == 0;  // always true by construction
 
   // Each warpgroup executes one register-split instruction (one site per
@@ -513,13 +558,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t s_cnt = 0;      // S_t completions consumed so far (all pieces)
     uint32_t piece_cnt = 0;  // pieces finished
     bool ok = true;
-    while (ok && pit.next(p, pc)) {
+    while (ok && pit.next(p, pc, unit_plan)) {
       const int ntt = t ? pc.a1 : pc.a0;
       const int r0t = pc.qb * kRowsPerCta + t * kBlockM;
       const int row = r0t + rt;
-      float m_raw = -INFINITY;  // running max of the raw scores
+      float m_raw = -INFINITY;  // reference max of the raw scores (-inf while no key was visible)
       float m_sc = 0.f;         // m_raw * c (0 while no key was visible)
       float l = 0.f;            // running denominator, relative to m_sc
+      float lr = 0.f;           // bf16 rounding of each tile's largest probability, summed like l
       for (int jj = 0; jj < ntt; ++jj) {
         const int j = pc.j0 + pc.jb + jj;  // K/V tile (absolute)
         if (!mbar_wait_warp(bar(BAR_S + t), s_cnt & 1, g, FA2_SITE_S_READY, j)) {
@@ -564,13 +610,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 16; i < kBlockN; i += 16)
 #pragma unroll
           for (int k = 0; k < 8; ++k) mp[k] = fmax3(mp[k], s[i + 2 * k], s[i + 2 * k + 1]);
-        const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]),
-                               fmax3(mp[6], mp[7], m_raw));
-        const float m_sc_new = (mx == -INFINITY) ? 0.f : mx * c;
-        // rescale factor for what was accumulated so far: exactly 1 when the max
-        // did not move (then O is left untouched), 0 when nothing was visible yet
-        float alpha = 1.f;
-        if (mx != m_raw) alpha = (m_raw == -INFINITY) ? 0.f : ex2_approx(m_sc - m_sc_new);
+        const float tmx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
+        const float mx = fmaxf(tmx, m_raw);
+        // New reference: the running max, taken when nothing was visible yet or
+        // when it exceeds the current reference by more than the threshold;
+        // otherwise the reference stays and the rescale factor is exactly 1 (O
+        // is left untouched).  alpha is 0 when nothing was visible yet.
+        float m_ref = m_raw, m_sc_new = m_sc, alpha = 1.f;
+        if (m_raw == -INFINITY) {
+          if (mx != -INFINITY) {
+            m_ref = mx;
+            m_sc_new = mx * c;
+            alpha = 0.f;
+          }
+        } else if (mx * c - m_sc > kRescaleThreshold) {
+          m_ref = mx;
+          m_sc_new = mx * c;
+          alpha = ex2_approx(m_sc - m_sc_new);
+        }
         if (jj > 0) {
           // Publish the rescale factor; the correction warps apply it to O
           // while this thread computes the exponentials.
@@ -601,6 +658,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               pk[i] = pack_bf16x2(e0, e1);
             }
             tmem_st16(tP + 16 * k, pk);
+            if (k == 1) {
+              // keys 0-63 of P are in TMEM: the first half of the PV product
+              // can start while the second half is computed
+              tmem_wait_st();
+              tc_fence_before();
+              mbar_arrive(bar(BAR_PH + t));
+            }
           }
         };
         if (masked)  // masked scores are -inf and must give exactly 0: MUFU only
@@ -614,7 +678,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(BAR_P + t));
         l = l * alpha + (((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7])));
-        m_raw = mx;
+        {
+          // the tile's largest probability as the PV product saw it (bf16) minus
+          // its fp32 value, computed with the same fused multiply-add and exp2
+          const float pm = (tmx == -INFINITY) ? 0.f : ex2_approx(fmaf(tmx, c, -m_sc_new));
+          const float rm = __uint_as_float(pack_bf16x2(pm, 0.f) << 16);
+          lr = lr * alpha + (rm - pm);
+        }
+        m_raw = m_ref;
         m_sc = m_sc_new;
       }
       if (!ok) break;
@@ -626,6 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       sm_m[t * kBlockM + rt] = (m_raw == -INFINITY) ? -INFINITY : m_sc;
       sm_l[t * kBlockM + rt] = l;
+      sm_lr[t * kBlockM + rt] = lr;
       mbar_arrive(bar(BAR_FSTATS + t));
       ++piece_cnt;
     }
@@ -643,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ph = 0;
     bool ok = true;
 
-    while (ok && pit.next(p, pc)) {
+    while (ok && pit.next(p, pc, unit_plan)) {
       const int n_p = pc.je - pc.jb;
       for (int jj = 0; jj < n_p && ok; ++jj) {
 #pragma unroll
@@ -651,7 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (jj >= (t ? pc.a1 : pc.a0)) continue;
           if (jj == 0) {  // nothing accumulated yet: O_t (read by the last epilogue) is free
             tc_fence_before();
-            mbar_arrive(bar(BAR_P + t));
+            mbar_arrive(bar(BAR_PH + t));
             continue;
           }
           if (!mbar_wait_warp(bar(BAR_STATS + t), (ph >> t) & 1, g, FA2_SITE_STATS_READY, pc.jb + jj)) {
@@ -683,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_st();
           }
           tc_fence_before();
-          mbar_arrive(bar(BAR_P + t));
+          mbar_arrive(bar(BAR_PH + t));
         }
       }
       if (!ok) break;
@@ -712,6 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float m_sc = sm_m[t * kBlockM + rt];
         const float l = sm_l[t * kBlockM + rt];
+        const float lr = sm_lr[t * kBlockM + rt];
         mbar_arrive(bar(BAR_FCONS + t));
         tc_fence_after();
         const uint32_t tO = tmem + lane_off + C::col_o(t);
@@ -721,7 +794,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool valid = row < p.Nq;
           float inv_l = 0.f, lse = -INFINITY;
           if (l > 0.f) {
-            inv_l = 1.f / l;
+            inv_l = 1.f / (l + lr);
             lse = (m_sc + log2f(l)) * 0.69314718055994530942f;
           }
           __nv_bfloat16* orow = p.o + ((static_cast<size_t>(pc.b) * p.Nq + row) * p.Hq + pc.hq) * D;
@@ -769,6 +842,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __stcg(part + C::part_m(t, rt), m_sc);
           __stcg(part + C::part_l(t, rt), have ? l : 0.f);
+          __stcg(part + C::part_lr(t, rt), have ? lr : 0.f);
         }
       }
       if (!ok) break;
@@ -832,15 +906,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       };
-      // O_t (+)= P_t V with the V tile of ring item itV, then commits
-      auto issue_pv = [&](int t, uint32_t itV, bool acc, uint32_t c1, uint32_t c2) {
+      // O_t (+)= P_t V over keys [16 k0, 16 k1) of the V tile of ring item itV, then commits
+      auto issue_pv = [&](int t, uint32_t itV, bool acc, int k0, int k1, uint32_t c1, uint32_t c2) {
         const uint32_t dS = tmem + C::col_s(t), dO = tmem + C::col_o(t);
         const uint64_t bV = dV + ((stage_of(itV) * C::kTileBytes) >> 4);
         if (elect_one()) {
-          uint64_t db = bV;
+          uint64_t db = bV + static_cast<uint32_t>(k0) * ((16 * kSwizzleBytes) >> 4);
           asm volatile("" : "+l"(db));
 #pragma unroll
-          for (int kk = 0; kk < kBlockN / 16; ++kk) {
+          for (int kk = k0; kk < k1; ++kk) {
             umma_ts(dO, dS + kk * 8, db, idPV, (acc || kk > 0) ? 1u : 0u);
             db += (16 * kSwizzleBytes) >> 4;  // next 16 keys
           }
@@ -853,7 +927,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t q_cnt = 0;         // pieces whose Q was waited for
       uint32_t p_cnt[2] = {0, 0}; // P_t phases consumed
       bool ok = true;
-      while (ok && pit.next(p, pc)) {
+      while (ok && pit.next(p, pc, unit_plan)) {
         const int n_p = pc.je - pc.jb;
         const int a0 = pc.a0, a1 = pc.a1;
         if (!mbar_wait_warp(bar(BAR_Q), q_cnt & 1, g, FA2_SITE_Q_LOADED, q_cnt)) break;
@@ -883,10 +957,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t qfree = (SK && jj + 2 == n_p) ? bar(BAR_QFREE) : 0u;
           // tile 0: PV0(j) and S0(j+1); V_j / K_{j+1} are freed here when tile 1 has no use for them
           if (jj < a0) {
+            // keys 0-63 as soon as their P is written and O_0 is rescaled, then the rest
+            if (!mbar_wait_warp(bar(BAR_PH + 0), p_cnt[0] & 1, g, FA2_SITE_O_RESCALED, pc.jb + jj)) break;
+            tc_fence_after();
+            issue_pv(0, itV(jj), jj > 0, 0, kBlockN / 32, 0u, 0u);
             if (!mbar_wait_warp(bar(BAR_P + 0), p_cnt[0] & 1, g, FA2_SITE_P_READY, pc.jb + jj)) break;
             ++p_cnt[0];
             tc_fence_after();
-            issue_pv(0, itV(jj), jj > 0, jj == a0 - 1 ? bar(BAR_OFINAL + 0) : 0u,
+            issue_pv(0, itV(jj), true, kBlockN / 32, kBlockN / 16, jj == a0 - 1 ? bar(BAR_OFINAL + 0) : 0u,
                      jj >= a1 ? free_of(itV(jj)) : 0u);
             if (jj + 1 < a0)
               issue_s(0, itK(jj + 1), bar(BAR_S + 0), jj + 1 >= a1 ? free_of(itK(jj + 1)) : 0u,
@@ -894,10 +972,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           // tile 1: PV1(j) and S1(j+1); the last use of V_j and K_{j+1}
           if (jj < a1) {
+            if (!mbar_wait_warp(bar(BAR_PH + 1), p_cnt[1] & 1, g, FA2_SITE_O_RESCALED, pc.jb + jj)) break;
+            tc_fence_after();
+            issue_pv(1, itV(jj), jj > 0, 0, kBlockN / 32, 0u, 0u);
             if (!mbar_wait_warp(bar(BAR_P + 1), p_cnt[1] & 1, g, FA2_SITE_P_READY, pc.jb + jj)) break;
             ++p_cnt[1];
             tc_fence_after();
-            issue_pv(1, itV(jj), jj > 0, free_of(itV(jj)), jj == a1 - 1 ? bar(BAR_OFINAL + 1) : 0u);
+            issue_pv(1, itV(jj), true, kBlockN / 32, kBlockN / 16, free_of(itV(jj)),
+                     jj == a1 - 1 ? bar(BAR_OFINAL + 1) : 0u);
             if (jj + 1 < a1) issue_s(1, itK(jj + 1), bar(BAR_S + 1), free_of(itK(jj + 1)), qfree);
           }
         }
@@ -917,7 +999,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;       // ring items issued
       uint32_t pieces = 0;   // pieces whose Q was loaded
       bool ok = true;
-      while (ok && pit.next(p, pc)) {
+      while (ok && pit.next(p, pc, unit_plan)) {
         const int hk = pc.hq / (p.Hq / p.Hkv);
         // Q of this piece, once the previous piece's last S MMA released the buffer
         if (pieces > 0 && !mbar_wait_warp(bar(BAR_QFREE), (pieces - 1) & 1, g, FA2_SITE_Q_LOADED, pieces)) {
@@ -1060,16 +1142,17 @@ __global__ void __launch_bounds__(kCombineThreads) fa2_combine_kernel(const Para
     for (int i = 0; i < kBatch; ++i)
       if (lq[i] > 0.f) m_tot = fmaxf(m_tot, mq[i]);
   }
-  float l_tot = 0.f;
+  float l_tot = 0.f, lr_tot = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int q0 = 0; q0 < np; q0 += kBatch) {
-    float mq[kBatch], lq[kBatch];
+    float mq[kBatch], lq[kBatch], lrq[kBatch];
     float4 f[kBatch];
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
       const bool in = q0 + i < np;
       const float* base = part(in ? q0 + i : q0);
       lq[i] = in ? __ldcg(base + C::part_l(t, rt)) : 0.f;
+      lrq[i] = __ldcg(base + C::part_lr(t, rt));
       mq[i] = __ldcg(base + C::part_m(t, rt));
       // a piece with l = 0 may not have written its O: loaded, then skipped
       f[i] = __ldcg(reinterpret_cast<const float4*>(base + C::part_o(t, ch, rt)) + f4);
@@ -1079,13 +1162,14 @@ __global__ void __launch_bounds__(kCombineThreads) fa2_combine_kernel(const Para
       if (!(lq[i] > 0.f)) continue;
       const float wq = ex2_approx(mq[i] - m_tot);
       l_tot = fmaf(lq[i], wq, l_tot);
+      lr_tot = fmaf(lrq[i], wq, lr_tot);
       acc.x = fmaf(wq, f[i].x, acc.x);
       acc.y = fmaf(wq, f[i].y, acc.y);
       acc.z = fmaf(wq, f[i].z, acc.z);
       acc.w = fmaf(wq, f[i].w, acc.w);
     }
   }
-  const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
+  const float inv_l = (l_tot > 0.f) ? 1.f / (l_tot + lr_tot) : 0.f;
   __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Nq + row) * p.Hq + hq) * D;
   uint2 o2;
   o2.x = pack_bf16x2(acc.x * inv_l, acc.y * inv_l);
@@ -1193,9 +1277,65 @@ static Plan make_plan(int B, int Hq, int Nq, int Nk, Window win, int d, int num_
   pl.G = static_cast<int>(pl.iters < num_sms ? pl.iters : num_sms);
   // a CTA's range holds at most two pieces of split units (its first and its
   // last), so two partial buffers per CTA cover every split
-  const long long piece_bytes = 4LL * kTiles * kBlockM * (d + 2);
+  const long long piece_bytes = 4LL * kTiles * kBlockM * (d + 3);
   pl.ws_bytes = (pl.G > 1) ? 2LL * pl.G * piece_bytes : 0;
   return pl;
+}
+
+// Plan of persistent whole units (UnitTable).  The heavier units are listed in
+// groups of consecutive (batch, head) pairs -- whole GQA groups, about one
+// wave of units per group -- heaviest first inside each group; the light
+// units (at most 40 % of the heaviest unit's cost) follow, across all heads,
+// heaviest first.  Each unit in turn goes to the CTA whose planned work (K/V
+// tile iterations plus the fixed cost of a unit) is smallest.  The groups keep
+// the CTAs running at any moment on a few neighbouring heads, whose K and V
+// then stay in L2; the light tail evens out the CTAs' work at the end, where a
+// purely head-ordered list would leave some heavy units last ("FlashAttention
+// 2: Three Places the Chip Was Still Waiting", section 2.3: many more blocks
+// than SMs; which of them share the cache is this library's choice).  Returns
+// false when the problem exceeds the table.
+static bool plan_units(int B, int Hq, int Hkv, int Nq, int Nk, Window win, int n_qblk, int r_empty,
+                       int G, UnitTable& tab) {
+  const long long HB = static_cast<long long>(B) * Hq;
+  const long long units = HB * r_empty;
+  if (G <= 0 || G > kMaxTableCtas || units <= 0 || units > kMaxTableUnits) return false;
+  const int grp = Hq / Hkv;  // query heads sharing a KV head
+  // heads per group: about one wave of units, a whole number of GQA groups
+  long long hg = (static_cast<long long>(G) + r_empty - 1) / r_empty;
+  hg = ((hg + grp - 1) / grp) * grp;
+  if (hg > HB) hg = HB;
+  std::vector<int> cost(r_empty);
+  int cmax = 0;
+  for (int r = 0; r < r_empty; ++r) {
+    cost[r] = unit_tiles(Nq, Nk, win, n_qblk - 1 - r) + kUnitCost;
+    cmax = std::max(cmax, cost[r]);
+  }
+  std::vector<int> heavy, light;  // rounds
+  for (int r = 0; r < r_empty; ++r) (5 * cost[r] > 2 * cmax ? heavy : light).push_back(r);
+  std::stable_sort(light.begin(), light.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+  // list scheduling: the next unit goes to the CTA with the least planned work
+  using Slot = std::pair<long long, int>;  // (planned work, CTA)
+  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> free_at;
+  for (int c = 0; c < G; ++c) free_at.push({0, c});
+  std::vector<std::vector<uint16_t>> lists(G);
+  auto assign = [&](int r, long long k) {
+    const Slot sl = free_at.top();
+    free_at.pop();
+    lists[sl.second].push_back(static_cast<uint16_t>(r * HB + k));
+    free_at.push({sl.first + cost[r], sl.second});
+  };
+  for (long long k0 = 0; k0 < HB; k0 += hg)
+    for (int r : heavy)
+      for (long long k = k0; k < std::min(HB, k0 + hg); ++k) assign(r, k);
+  for (int r : light)
+    for (long long k = 0; k < HB; ++k) assign(r, k);
+  int pos = 0;
+  for (int c = 0; c < G; ++c) {
+    tab.start[c] = static_cast<uint16_t>(pos);
+    for (uint16_t u : lists[c]) tab.unit[pos++] = u;
+  }
+  tab.start[G] = static_cast<uint16_t>(pos);
+  return true;
 }
 
 static int sm_count() {
@@ -1228,7 +1368,7 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
   static std::once_flag flags[kMaxDevices];
   static int setup_status[kMaxDevices];
   const int st = once_per_device(flags, setup_status, [] {
-    for (auto* kern : {fa2_fwd_kernel<D, false>, fa2_fwd_kernel<D, true>}) {
+    auto setup = [](auto* kern) {
       cudaFuncAttributes attr;
       if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return static_cast<int>(FA2_ERR_LAUNCH);
       // the setmaxnreg split assumes exactly this pool
@@ -1236,8 +1376,10 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
           cudaSuccess)
         return static_cast<int>(FA2_ERR_LAUNCH);
-    }
-    return static_cast<int>(FA2_OK);
+      return static_cast<int>(FA2_OK);
+    };
+    const int s0 = setup(fa2_fwd_kernel<D, false>);
+    return s0 != FA2_OK ? s0 : setup(fa2_fwd_kernel<D, true>);
   });
   if (st != FA2_OK) return st;
 
@@ -1262,6 +1404,7 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
   p.limit_ns = 1000000000u;  // 1 s per wait; a healthy wait takes microseconds
   p.streamk = 0;
   p.pu = 0;
+  p.tab = 0;
   p.T = 0;
   p.span = 0;
   p.rem = 0;
@@ -1270,12 +1413,14 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
   unsigned grid = static_cast<unsigned>(p.n_qblk) * Hq * B;  // one unit per CTA
   const long long units_ne = static_cast<long long>(p.r_empty) * Hq * B;
   const int sms = sm_count();
+  static thread_local UnitTable plan;  // kernel parameter of the persistent launch
   if (!workspace && persistent_units && sms > 0 && units_ne >= 2LL * sms) {
     // persistent CTAs over whole units: the next unit's Q and K/V stream in
     // while the current one drains, instead of a block exit and launch
     p.pu = 1;
     p.G = sms;
     grid = static_cast<unsigned>(sms);
+    p.tab = plan_units(B, Hq, Hkv, Nq, Nk, win, p.n_qblk, p.r_empty, sms, plan) ? 1 : 0;
   }
   if (workspace) {
     const Plan pl = make_plan(B, Hq, Nq, Nk, win, D, sm_count());
@@ -1297,9 +1442,9 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
       !encode_bnhd(&tv, v, B, Nk, Hkv, D))
     return FA2_ERR_LAUNCH;
   if (p.streamk || p.pu)
-    fa2_fwd_kernel<D, true><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+    fa2_fwd_kernel<D, true><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p, plan);
   else
-    fa2_fwd_kernel<D, false><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+    fa2_fwd_kernel<D, false><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p, NoTable{});
   if (cudaGetLastError() != cudaSuccess) return FA2_ERR_LAUNCH;
   if (p.streamk && p.G > 1) {
     const dim3 cgrid(static_cast<unsigned>(p.G - 1), kRowsPerCta / kCombineRows, D / 16);
@@ -1456,7 +1601,7 @@ extern "C" int fa2_forward_ws(const void* q, const void* k, const void* v, void*
 // same call.  One array per device serves every call, so calls that may
 // overlap in time race on it.
 // ---------------------------------------------------------------------------
-constexpr size_t kStaticScratchBytes = FA2_STATIC_WS_BYTES;  // 2 partials x 148 SMs at d = 128 fit
+constexpr size_t kStaticScratchBytes = FA2_STATIC_WS_BYTES;  // 2 partials x 156 SMs at d = 128 fit
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 // Device address of the array on device `dev` (the current device), or
@@ -1550,6 +1695,24 @@ extern "C" long long fa2_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, 
   if (n <= 0) return -1;
   const Plan pl = make_plan(B, Hq, Nq, Nk, causal_window(causal), d, n);
   return pl.T > INT_MAX ? -1 : pl.ws_bytes;
+}
+
+extern "C" int fa2_persistent_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                                   int num_sms, int* start, int* units, int units_capacity) {
+  const int sv = validate_shape(B, Hq, Hkv, Nq, Nk, d);
+  if (sv != FA2_OK) return sv;
+  if (!start || !units) return FA2_ERR_NULL_POINTER;
+  if (num_sms <= 0) return FA2_ERR_BAD_SHAPE;
+  const Window win = causal_window(causal);
+  const int n_qblk = (Nq + kRowsPerCta - 1) / kRowsPerCta;
+  int r_empty = 0;
+  while (r_empty < n_qblk && unit_tiles(Nq, Nk, win, n_qblk - 1 - r_empty) > 0) ++r_empty;
+  static thread_local UnitTable tab;
+  if (!plan_units(B, Hq, Hkv, Nq, Nk, win, n_qblk, r_empty, num_sms, tab)) return FA2_ERR_SIZE;
+  if (tab.start[num_sms] > units_capacity) return FA2_ERR_SIZE;
+  for (int c = 0; c <= num_sms; ++c) start[c] = tab.start[c];
+  for (int i = 0; i < tab.start[num_sms]; ++i) units[i] = tab.unit[i];
+  return FA2_OK;
 }
 
 extern "C" int fa2_streamk_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,

@@ -150,7 +150,7 @@ int fa2_forward_ws(const void* q, const void* k, const void* v, void* o, float* 
 
 /*
  * fa2_workspace_size -- bytes of workspace fa2_forward_ws needs for this
- * problem on the current device: two partials of 2 x 128 x (d + 2) floats per
+ * problem on the current device: two partials of 2 x 128 x (d + 3) floats per
  * SM (0 when the work fits one block).  Returns -1 for an invalid shape (as fa2_forward validates it),
  * for a problem fa2_forward_ws refuses with FA2_ERR_SIZE, or when the device
  * cannot be queried.  Queries the device's SM count; makes no
@@ -174,7 +174,7 @@ long long fa2_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int 
  * Nothing in the array needs to start at zero: every partial the merge reads
  * is written earlier in the same call.  Returns FA2_ERR_WORKSPACE when the
  * problem's fa2_workspace_size exceeds FA2_STATIC_WS_BYTES (it fits for
- * d = 64 and d = 128 on GPUs with up to 157 SMs), FA2_ERR_LAUNCH when the
+ * d = 64 and d = 128 on GPUs with up to 156 SMs), FA2_ERR_LAUNCH when the
  * array's device address cannot be obtained, and otherwise what
  * fa2_forward_ws returns.
  *
@@ -289,13 +289,37 @@ int fa2_selftest_timeout(void* stream, long long limit_ns);
  * fa2_launch_plan: the work decomposition fa2_forward uses for a problem:
  * the number of units (256 query rows of one head and batch each, one thread
  * block apiece when there are fewer than two units per SM; otherwise one
- * persistent block per SM takes whole units round robin, heaviest first),
+ * persistent block per SM takes whole units, see fa2_persistent_plan),
  * threads per block, dynamic shared memory bytes and query rows per unit.
  * Returns an fa2_status_code (validation as in fa2_forward, minus pointers).
  */
 long long fa2_num_blocks(int B, int H, int N, int rows_per_block);
 int fa2_launch_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int* grid_blocks,
                     int* threads_per_block, int* smem_bytes, int* rows_per_block);
+
+/*
+ * fa2_persistent_plan: which units the persistent blocks of fa2_forward run,
+ * in which order, on a GPU with num_sms SMs (fa2_forward uses it when the
+ * problem has at least two units with a visible key per SM).  Units are
+ * grouped by neighbouring (batch, head) pairs -- whole GQA groups, about one
+ * wave of units per group -- heaviest first inside a group, and each goes to
+ * the block with the least planned work (K/V tiles plus a fixed cost per
+ * unit), so that the blocks running at any moment share a few heads' K and V
+ * in L2 ("FlashAttention 2: Three Places the Chip Was Still Waiting",
+ * section 2.3 for the units; the order is this library's).  The plan is a
+ * kernel parameter: nothing is allocated.
+ *
+ *   start   num_sms + 1 ints (host): block c runs units[start[c] .. start[c+1])
+ *   units   units_capacity ints (host): unit u = round * B * Hq + b * Hq + hq,
+ *           round = query blocks counted from the last
+ *
+ * Returns FA2_OK; FA2_ERR_SIZE when the problem has more than 8192 units with
+ * a visible key, num_sms exceeds 160 (fa2_forward then deals units round
+ * robin, heaviest first) or units_capacity is too small; FA2_ERR_NULL_POINTER
+ * for missing arrays; otherwise fa2_forward's validation status.  No CUDA call.
+ */
+int fa2_persistent_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, int num_sms,
+                        int* start, int* units, int units_capacity);
 
 /*
  * fa2_streamk_plan: the stream-K schedule fa2_forward_ws would use on a GPU

@@ -41,11 +41,11 @@ def test_static_validation_before_any_cuda_call():
 
 
 def test_static_capacity_covers_this_gpu_class():
-    # two fp32 partials of 2 x 128 x (d + 2) floats per SM: 157 SMs fit at d = 128, 158 do not
+    # two fp32 partials of 2 x 128 x (d + 3) floats per SM: 156 SMs fit at d = 128, 157 do not
     for d in (64, 128):
-        st, _, G, ws = fa2.fa2_streamk_plan(1, 1, 1, 256, 1 << 20, d, 0, 157)
-        assert st == 0 and G == 157 and ws <= fa2.FA2_STATIC_WS_BYTES
-    st, _, G, ws = fa2.fa2_streamk_plan(1, 1, 1, 256, 1 << 20, 128, 0, 158)
+        st, _, G, ws = fa2.fa2_streamk_plan(1, 1, 1, 256, 1 << 20, d, 0, 156)
+        assert st == 0 and G == 156 and ws <= fa2.FA2_STATIC_WS_BYTES
+    st, _, G, ws = fa2.fa2_streamk_plan(1, 1, 1, 256, 1 << 20, 128, 0, 157)
     assert st == 0 and ws > fa2.FA2_STATIC_WS_BYTES
 
 

@@ -478,9 +478,11 @@ __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& e0, fl
 
 // Pairs of each 32-column chunk whose exponentials go through exp2_poly_pair
 // in unmasked tiles (the rest use the MUFU).  It moves work from the MUFU to
-// the FMA pipe; measured on B200 it does not pay while the per-tile chain,
-// not MUFU throughput, bounds the kernel (2 or 4 pairs: -4 to -8 % on causal
-// 8k), so the default is 0.
+// the FMA pipe.  Measured on B200 with the final kernel (interleaved runs,
+// 2 of 16 pairs): within +-1 % on causal 8k, non-causal 2k, GQA 4k and long
+// 32k, because the exponentials are not what bounds the per-tile chain (a
+// timing probe without any exponential is only ~5 % faster); the default is
+// 0.  Built and checked against the oracle with 2 pairs by the GPU tests.
 #ifndef FA2_EMU_PAIRS
 #define FA2_EMU_PAIRS 0
 #endif

@@ -1458,64 +1458,6 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
 
 #include "fa2_backward.cuh"
 
-template <int D>
-static int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                      const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
-                      int Nk, Window win, float scale, void* workspace, cudaStream_t stream) {
-  using C = BCfg<D>;
-  static std::once_flag flags[kMaxDevices];
-  static int setup_status[kMaxDevices];
-  const int st = once_per_device(flags, setup_status, [] {
-    return cudaFuncSetAttribute(fa2_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                C::kSmemBytes) == cudaSuccess
-               ? static_cast<int>(FA2_OK)
-               : static_cast<int>(FA2_ERR_LAUNCH);
-  });
-  if (st != FA2_OK) return st;
-  const long long rows = static_cast<long long>(B) * Nq * Hq;
-  float* dq_acc = static_cast<float*>(workspace);
-  float* lse2 = dq_acc + ((rows * D + 63) / 64) * 64;
-  float* delta = lse2 + ((rows + 63) / 64) * 64;
-  fa2_bwd_prep_kernel<D><<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
-      dq_acc, B, Hq, Nq);
-  if (cudaGetLastError() != cudaSuccess) return FA2_ERR_LAUNCH;
-  CUtensorMap tq, tk, tv, tdo;
-  if (!encode_bnhd(&tq, q, B, Nq, Hq, D) || !encode_bnhd(&tk, k, B, Nk, Hkv, D) ||
-      !encode_bnhd(&tv, v, B, Nk, Hkv, D) || !encode_bnhd(&tdo, dout, B, Nq, Hq, D))
-    return FA2_ERR_LAUNCH;
-  BwdParams p;
-  p.lse2 = lse2;
-  p.delta = delta;
-  p.dq_acc = dq_acc;
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.Nq = Nq;
-  p.Nk = Nk;
-  p.wl = win.wl;
-  p.wr = win.wr;
-  p.scale = scale;
-  p.c = scale * 1.4426950408889634f;
-  p.limit_ns = 1000000000u;
-  const dim3 grid(static_cast<unsigned>((Nk + kBlockN - 1) / kBlockN), Hkv, B);
-  fa2_bwd_kernel<D><<<grid, kBwdThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
-  if (cudaGetLastError() != cudaSuccess) return FA2_ERR_LAUNCH;
-  const long long n4 = rows * D / 4;
-  fa2_bwd_dq_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(
-      dq_acc, static_cast<__nv_bfloat16*>(dq), n4);
-  return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_LAUNCH;
-}
-
-// Bytes of backward workspace: the fp32 dQ accumulator, then LSE in log2
-// units and D per row (each region rounded up to 64 floats).
-static long long bwd_workspace_bytes(int B, int Hq, int Nq, int d) {
-  const long long rows = static_cast<long long>(B) * Nq * Hq;
-  return 4LL * (((rows * d + 63) / 64) * 64 + 2 * ((rows + 63) / 64) * 64);
-}
-
 static int check_device() {
   static std::once_flag flags[kMaxDevices];
   static int cached[kMaxDevices];

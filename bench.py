@@ -431,6 +431,8 @@ def run_fa2(args, w):
         n_e2e = max(3, min(args.steps, 50))
         h2d_stream, d2h_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         chunks = w.B
+        if chunks == 1:  # nothing to overlap: one stream, as a caller would
+            h2d_stream = d2h_stream = stream
 
         def call_b(b, qq, kk, vv, oo, ll):
             if w.windowed:

@@ -79,7 +79,9 @@ enum Bar {
   BAR_FCONS = 12,    // [2] final statistics read by the epilogue (128 correction threads)
   BAR_DONE = 14,     // all MMAs drained (MMA commit)
   BAR_PH = 15,       // [2] keys 0-63 of P written and O rescaled (128 softmax + 128 correction threads)
-  BAR_KV_FULL = 17,  // [stages] K/V tile landed (TMA tx); then [stages] slot free (MMA commit)
+  BAR_K0 = 17,       // the first K tile of a piece landed (TMA tx)
+  BAR_KV_FULL = 18,  // [stages] a V slot's barrier: V_j and K_{j+1} landed (TMA tx; K slots' are
+                     // unused); then [stages] slot free (MMA commit)
 };
 
 // Scheduling cost of a unit, in K/V-tile iterations, on top of its
@@ -121,6 +123,13 @@ struct UnitTable {
   uint16_t unit[kMaxTableUnits];      // unit index u = round * B * Hq + (b * Hq + hq)
 };
 struct NoTable {};
+
+// Range boundaries of a stream-K launch that are the first cut of a split
+// unit: the combine kernel runs one block row per entry.
+struct CutList {
+  int n;
+  uint16_t c[kMaxTableCtas];
+};
 
 // Warps 14-15 (otherwise idle) write the rows of units with no visible key.
 constexpr int kEmptyThreads = 64;
@@ -937,23 +946,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto itK = [&](int jj) { return itb + 2u * static_cast<uint32_t>(jj); };
         auto itV = [&](int jj) { return itb + 2u * static_cast<uint32_t>(jj) + 1u; };
         // S_t of the piece's first K/V tile; K is free after the last S on it
-        if (!mbar_wait_warp(bar(BAR_KV_FULL + stage_of(itK(0))), phase_of(itK(0)), g,
-                            FA2_SITE_KV_LOADED, pc.jb))
-          break;
+        if (!mbar_wait_warp(bar(BAR_K0), (q_cnt - 1) & 1, g, FA2_SITE_KV_LOADED, pc.jb)) break;
         tc_fence_after();
         // (one piece per CTA in unit mode: the Q buffer is never reloaded)
         const uint32_t qfree0 = (SK && n_p == 1) ? bar(BAR_QFREE) : 0u;
         if (a0 > 0) issue_s(0, itK(0), bar(BAR_S + 0), a1 > 0 ? 0u : free_of(itK(0)), a1 > 0 ? 0u : qfree0);
         if (a1 > 0) issue_s(1, itK(0), bar(BAR_S + 1), free_of(itK(0)), qfree0);
         for (int jj = 0; jj < n_p && ok; ++jj) {
-          const bool next = (jj + 1 < n_p);
-          // operands of this step (normally landed long ago); checked while the
-          // tensor pipe still holds the previous block
+          // operands of this step, V_j and K_{j+1}, behind one barrier (V_j's);
+          // checked while the tensor pipe still holds the previous block
           if (!mbar_wait_warp(bar(BAR_KV_FULL + stage_of(itV(jj))), phase_of(itV(jj)), g,
                               FA2_SITE_KV_LOADED, pc.jb + jj))
-            break;
-          if (next && !mbar_wait_warp(bar(BAR_KV_FULL + stage_of(itK(jj + 1))), phase_of(itK(jj + 1)), g,
-                                      FA2_SITE_KV_LOADED, pc.jb + jj + 1))
             break;
           // the last S of the piece frees the Q buffer for the next piece
           const uint32_t qfree = (SK && jj + 2 == n_p) ? bar(BAR_QFREE) : 0u;
@@ -1022,6 +1025,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         ++pieces;
+        // Ring items K_0, V_0, K_1, V_1, ...: K_0 signals BAR_K0; V_j and K_{j+1}
+        // (what the MMA step j needs) both signal V_j's barrier, so the MMA
+        // warp waits once per step.
+        uint32_t vbar = 0;  // barrier of the last V item
         for (int j = pc.j0 + pc.jb; j < pc.j0 + pc.je && ok; ++j) {  // absolute K/V tiles
 #pragma unroll 1
           for (int kv = 0; kv < 2; ++kv, ++it) {
@@ -1032,13 +1039,23 @@ __global__ void __launch_bounds__(kThreads, 1)
               ok = false;
               break;
             }
+            const bool first_k = (kv == 0 && j == pc.j0 + pc.jb);
+            uint32_t tb;
+            if (kv == 1) {
+              vbar = bar(BAR_KV_FULL + st);
+              tb = vbar;
+            } else {
+              tb = first_k ? bar(BAR_K0) : vbar;
+            }
             if (elect_one()) {
-              mbar_arrive_expect_tx(bar(BAR_KV_FULL + st), C::kTileBytes);
+              if (kv == 1)
+                mbar_arrive_expect_tx(tb, (j + 1 < pc.j0 + pc.je ? 2 : 1) * C::kTileBytes);
+              else if (first_k)
+                mbar_arrive_expect_tx(tb, C::kTileBytes);
               const CUtensorMap* map = kv ? &tmV : &tmK;
 #pragma unroll
               for (int ch = 0; ch < C::kChunks; ++ch)
-                tma_load_4d(sKV + st * C::kTileBytes + ch * kChunkBytes, map, bar(BAR_KV_FULL + st),
-                            ch * 64, hk, j * kBlockN, pc.b);
+                tma_load_4d(sKV + st * C::kTileBytes + ch * kChunkBytes, map, tb, ch * 64, hk, j * kBlockN, pc.b);
             }
             __syncwarp();
           }
@@ -1048,8 +1065,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Give the copies already in flight time to land before the CTA exits.
         const WaitGuard drain{0u, p.limit_ns};
         for (uint32_t i = (it > static_cast<uint32_t>(C::kStages) ? it - C::kStages : 0u); i < it; ++i)
-          mbar_wait_warp(bar(BAR_KV_FULL + i % C::kStages), (i / C::kStages) & 1, drain,
-                         FA2_SITE_LOAD_DRAIN, static_cast<int>(i));
+          if (i & 1u)  // V items: their barrier also counts the next K tile
+            mbar_wait_warp(bar(BAR_KV_FULL + i % C::kStages), (i / C::kStages) & 1, drain,
+                           FA2_SITE_LOAD_DRAIN, static_cast<int>(i));
+        if (pieces > 0) mbar_wait_warp(bar(BAR_K0), (pieces - 1) & 1, drain, FA2_SITE_LOAD_DRAIN, 0);
         if (pieces > 0) mbar_wait_warp(bar(BAR_Q), (pieces - 1) & 1, drain, FA2_SITE_LOAD_DRAIN, 0);
       }
     }
@@ -1096,18 +1115,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 // in view" and "Another use of mergeable statistics").  Pieces are summed in
 // their order in the unit, so the result is deterministic.
 //
-// Grid: (boundary c = 1..G-1) x (64-row block of the unit's 256 rows) x
-// (16-column chunk of d).  The CTA of boundary c works only if B_c is the
-// first boundary inside some unit's iterations; 4 threads share a row, each
-// owning 4 consecutive columns, so a warp reads 512 contiguous bytes.
+// Grid: (boundary c that is the first cut of a split unit, listed by the
+// host) x (64-row block of the unit's 256 rows) x (16-column chunk of d);
+// 4 threads share a row, each owning 4 consecutive columns, so a warp reads
+// 512 contiguous bytes.
 // ---------------------------------------------------------------------------
 constexpr int kCombineThreads = 256;
 constexpr int kCombineRows = 64;
 
 template <int D>
-__global__ void __launch_bounds__(kCombineThreads) fa2_combine_kernel(const Params p) {
+__global__ void __launch_bounds__(kCombineThreads)
+    fa2_combine_kernel(const Params p, const __grid_constant__ CutList cuts) {
   using C = Cfg<D>;
-  const int c = static_cast<int>(blockIdx.x) + 1;
+  const int c = cuts.c[blockIdx.x];
   const int bc = range_start(p.span, p.rem, p.G, c);
   PieceIter<true> it;
   it.HB = p.B * p.Hq;
@@ -1130,39 +1150,49 @@ __global__ void __launch_bounds__(kCombineThreads) fa2_combine_kernel(const Para
   auto part = [&](int q) {
     return p.ws + static_cast<size_t>(2 * (slot + q) + (q == 0 ? 1 : 0)) * C::kPieceFloats;
   };
-  constexpr int kBatch = 4;  // loads of 4 pieces in flight before any is used
-  float m_tot = -INFINITY;
-  for (int q0 = 0; q0 < np; q0 += kBatch) {
-    float mq[kBatch], lq[kBatch];
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      const bool in = q0 + i < np;
-      lq[i] = in ? __ldcg(part(q0 + i) + C::part_l(t, rt)) : 0.f;
-      mq[i] = in ? __ldcg(part(q0 + i) + C::part_m(t, rt)) : -INFINITY;
-    }
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i)
-      if (lq[i] > 0.f) m_tot = fmaxf(m_tot, mq[i]);
-  }
-  float l_tot = 0.f, lr_tot = 0.f;
+  // One pass over the pieces in batches of kBatch, every load of a batch in
+  // flight at once (statistics and O together); the accumulator follows the
+  // running max across batches.  A unit has at most a few tens of pieces, so
+  // this is one or two round trips to memory per thread.
+  constexpr int kBatch = 8;
+  float m_run = -INFINITY, l_tot = 0.f, lr_tot = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int q0 = 0; q0 < np; q0 += kBatch) {
     float mq[kBatch], lq[kBatch], lrq[kBatch];
     float4 f[kBatch];
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
-      const bool in = q0 + i < np;
-      const float* base = part(in ? q0 + i : q0);
-      lq[i] = in ? __ldcg(base + C::part_l(t, rt)) : 0.f;
-      lrq[i] = __ldcg(base + C::part_lr(t, rt));
-      mq[i] = __ldcg(base + C::part_m(t, rt));
-      // a piece with l = 0 may not have written its O: loaded, then skipped
-      f[i] = __ldcg(reinterpret_cast<const float4*>(base + C::part_o(t, ch, rt)) + f4);
+      lq[i] = 0.f;
+      lrq[i] = 0.f;
+      mq[i] = -INFINITY;
+      f[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (q0 + i < np) {
+        const float* base = part(q0 + i);
+        lq[i] = __ldcg(base + C::part_l(t, rt));
+        lrq[i] = __ldcg(base + C::part_lr(t, rt));
+        mq[i] = __ldcg(base + C::part_m(t, rt));
+        // a piece with l = 0 may not have written its O: loaded, then skipped
+        f[i] = __ldcg(reinterpret_cast<const float4*>(base + C::part_o(t, ch, rt)) + f4);
+      }
+    }
+    float mb = m_run;
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i)
+      if (lq[i] > 0.f) mb = fmaxf(mb, mq[i]);
+    if (mb != m_run) {  // rescale what earlier batches accumulated
+      const float sc = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - mb);
+      l_tot *= sc;
+      lr_tot *= sc;
+      acc.x *= sc;
+      acc.y *= sc;
+      acc.z *= sc;
+      acc.w *= sc;
+      m_run = mb;
     }
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
       if (!(lq[i] > 0.f)) continue;
-      const float wq = ex2_approx(mq[i] - m_tot);
+      const float wq = ex2_approx(mq[i] - m_run);
       l_tot = fmaf(lq[i], wq, l_tot);
       lr_tot = fmaf(lrq[i], wq, lr_tot);
       acc.x = fmaf(wq, f[i].x, acc.x);
@@ -1171,6 +1201,7 @@ __global__ void __launch_bounds__(kCombineThreads) fa2_combine_kernel(const Para
       acc.w = fmaf(wq, f[i].w, acc.w);
     }
   }
+  const float m_tot = m_run;
   const float inv_l = (l_tot > 0.f) ? 1.f / (l_tot + lr_tot) : 0.f;
   __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Nq + row) * p.Hq + hq) * D;
   uint2 o2;
@@ -1340,6 +1371,34 @@ static bool plan_units(int B, int Hq, int Hkv, int Nq, int Nk, Window win, int n
   return true;
 }
 
+// The boundaries c (1 <= c < G) of a stream-K launch that cut a unit for the
+// first time, in the device's unit order (the same walk as PieceIter and the
+// combine kernel's own check).  False when G exceeds the list.
+static bool first_cuts(const Params& p, Window win, CutList& cuts) {
+  cuts.n = 0;
+  if (p.G - 1 > kMaxTableCtas) return false;
+  const long long HB = static_cast<long long>(p.B) * p.Hq;
+  auto cost = [](int n) { return n > 0 ? n + kUnitCost : 0; };
+  long long cum = 0;
+  int r = 0;
+  int n = unit_tiles(p.Nq, p.Nk, win, p.n_qblk - 1);
+  for (int c = 1; c < p.G; ++c) {
+    const long long bc = range_start(p.span, p.rem, p.G, c);
+    while (bc >= cum + HB * cost(n)) {  // boundaries increase with c: walk the rounds once
+      cum += HB * cost(n);
+      ++r;
+      n = unit_tiles(p.Nq, p.Nk, win, p.n_qblk - 1 - r);
+    }
+    const long long w = cost(n);
+    const long long k = (bc - cum) / w;
+    const long long s0 = cum + k * w + kUnitCost;
+    const bool cuts_unit = bc > s0 && bc <= s0 + n - 1;
+    const bool first = c == 1 || range_start(p.span, p.rem, p.G, c - 1) <= s0;
+    if (cuts_unit && first) cuts.c[cuts.n++] = static_cast<uint16_t>(c);
+  }
+  return true;
+}
+
 static int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -1449,9 +1508,13 @@ static int launch(const void* q, const void* k, const void* v, void* o, float* l
     fa2_fwd_kernel<D, false><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p, NoTable{});
   if (cudaGetLastError() != cudaSuccess) return FA2_ERR_LAUNCH;
   if (p.streamk && p.G > 1) {
-    const dim3 cgrid(static_cast<unsigned>(p.G - 1), kRowsPerCta / kCombineRows, D / 16);
-    fa2_combine_kernel<D><<<cgrid, kCombineThreads, 0, stream>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return FA2_ERR_LAUNCH;
+    CutList cuts;
+    if (!first_cuts(p, win, cuts)) return FA2_ERR_SIZE;
+    if (cuts.n > 0) {
+      const dim3 cgrid(static_cast<unsigned>(cuts.n), kRowsPerCta / kCombineRows, D / 16);
+      fa2_combine_kernel<D><<<cgrid, kCombineThreads, 0, stream>>>(p, cuts);
+      if (cudaGetLastError() != cudaSuccess) return FA2_ERR_LAUNCH;
+    }
   }
   return FA2_OK;
 }

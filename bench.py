@@ -431,8 +431,6 @@ def run_fa2(args, w):
         n_e2e = max(3, min(args.steps, 50))
         h2d_stream, d2h_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         chunks = w.B
-        if chunks == 1:  # nothing to overlap: one stream, as a caller would
-            h2d_stream = d2h_stream = stream
 
         def call_b(b, qq, kk, vv, oo, ll):
             if w.windowed:
@@ -448,23 +446,30 @@ def run_fa2(args, w):
             if st != 0:
                 raise fa2.FA2Error(st)
 
+        done_in = [torch.cuda.Event() for _ in range(chunks)]
+        done_out = [torch.cuda.Event() for _ in range(chunks)]
+
         def e2e_step():
-            done_in = []
+            if chunks == 1:  # one stream, in order, as a caller would
+                qd.copy_(qp, non_blocking=True)
+                kd.copy_(kp, non_blocking=True)
+                vd.copy_(vp, non_blocking=True)
+                call_b(0, qd, kd, vd, od, ld)
+                op.copy_(od, non_blocking=True)
+                lp.copy_(ld, non_blocking=True)
+                return
             with torch.cuda.stream(h2d_stream):
                 h2d_stream.wait_stream(stream)  # the previous step's kernels read these buffers
                 for b in range(chunks):
                     qd[b].copy_(qp[b], non_blocking=True)
                     kd[b].copy_(kp[b], non_blocking=True)
                     vd[b].copy_(vp[b], non_blocking=True)
-                    ev = torch.cuda.Event()
-                    ev.record(h2d_stream)
-                    done_in.append(ev)
+                    done_in[b].record(h2d_stream)
             for b in range(chunks):
                 stream.wait_event(done_in[b])
                 call_b(b, qd[b], kd[b], vd[b], od[b], ld[b])
-                ev = torch.cuda.Event()
-                ev.record(stream)
-                d2h_stream.wait_event(ev)
+                done_out[b].record(stream)
+                d2h_stream.wait_event(done_out[b])
                 with torch.cuda.stream(d2h_stream):
                     op[b].copy_(od[b], non_blocking=True)
                     lp[b].copy_(ld[b], non_blocking=True)

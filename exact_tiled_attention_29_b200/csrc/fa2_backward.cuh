@@ -21,8 +21,10 @@
 // tile of every query head of its group that sees any of its keys, so dK and
 // dV need no atomics (GQA sums the group's heads in place).  dQ is the only
 // output shared between CTAs: each CTA adds its 128 x d contribution per
-// query tile into an fp32 accumulator with vector atomics, and a last kernel
-// scales nothing (scale is applied before the atomics) and rounds it to bf16.
+// query tile into an fp32 accumulator with TMA bulk reductions (the scaled
+// tile is staged in the shared-memory dS buffer once the dQ MMA has read it),
+// and a last kernel rounds the accumulator to bf16 (scale is applied before
+// the reduction).
 //
 // Per query tile (tensor memory: S^T | dP^T | dV | dK):
 //   MMA   S^T = K Q^T (SS), dP^T = V dO^T (SS)            -> "S ready"
@@ -32,8 +34,10 @@
 //   MMA   dV += P^T dO (TS), dK += dS^T Q (TS), dQ_tile = dS K (SS, into the
 //         S^T columns, after the dV MMA read P^T: one thread's MMAs run in
 //         issue order)                                     -> "dQ ready"
-//   WG0/1 read dQ_tile, scale, add into the fp32 accumulator -> "dQ free"
-//   and the next tile's S^T may overwrite the columns.
+//   WG0/1 read dQ_tile, scale          -> "dQ free": the next tile's S^T
+//         may overwrite the columns; stage the half tile in the dS buffer
+//         and one thread per warpgroup issues its bulk reduce-add into the
+//         fp32 accumulator; the next tile's dS waits for that read.
 //
 // Roles: warps 0-3 (WG0) and 4-7 (WG1) split the query columns of P / dS
 // (one thread per key row) and of the dQ read-out (one thread per query
@@ -41,6 +45,29 @@
 // register split: 384 threads leave 168 registers each.
 
 constexpr int kBwdThreads = 384;
+
+// 4-D tiled bulk reduction: adds one box of shared memory into global memory
+// (fp32 add, element-wise atomic with respect to other reductions), as part
+// of this thread's current bulk async-group.
+__device__ __forceinline__ void tma_reduce_add_4d(const void* map, uint32_t src, int c0, int c1, int c2,
+                                                  int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4, %5}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Every bulk operation this thread committed has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Every bulk operation this thread committed has completed.
+__device__ __forceinline__ void bulk_wait_group0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
 
 enum BwdBar {
   BB_KV = 0,        // K and V tiles of this CTA landed (TMA tx)
@@ -53,7 +80,9 @@ enum BwdBar {
   BB_DQ = 11,       // dQ tile complete
   BB_DQFREE = 12,   // dQ tile read out (128 WG1 threads)
   BB_DONE = 13,     // every MMA complete: dK, dV final
-  BB_COUNT = 14,
+  BB_STAGED = 14,   // [2] warpgroup wg's half of the dQ tile staged in the dS buffer (128 threads)
+  BB_STGREAD = 16,  // [2] warpgroup wg's bulk reduction has read the dS buffer (1 thread)
+  BB_COUNT = 18,
 };
 
 template <int D>
@@ -157,17 +186,12 @@ __global__ void __launch_bounds__(256) fa2_bwd_dq_kernel(const float* __restrict
   reinterpret_cast<uint2*>(dq)[idx] = w;
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
-}
 
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                   const BwdParams p) {
+                   const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using C = BCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -200,6 +224,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       uint32_t cnt = 1;
       if (i == BB_QFULL || i == BB_QFULL + 1) cnt = 32;
       if (i == BB_PDS || i == BB_DQFREE) cnt = 2 * kBlockM;
+      if (i == BB_STAGED || i == BB_STAGED + 1) cnt = kBlockM;
       mbar_init(bar(i), cnt);
     }
     fence_mbar_init();
@@ -213,6 +238,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmO);
+    tma_prefetch_desc(&tmDQ);
   }
   tc_fence_before();
   __syncthreads();
@@ -247,8 +273,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool masked = (q0 + kBlockM > p.Nq) || (k0 + kBlockN > p.Nk) ||
                           (p.wr >= 0 && k0 + kBlockN - 1 > q0 + koff + p.wr) ||
                           (p.wl >= 0 && k0 < q0 + kBlockM - 1 + koff - p.wl);
-      const float* lse_s = sm_lse + st * kBlockM;
-      const float* dl_s = sm_delta + st * kBlockM;
+      const uint32_t sL = sbase + C::kOffLse + 4u * st * kBlockM, sDl = sbase + C::kOffDelta + 4u * st * kBlockM;
 #pragma unroll 1
       for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
         uint32_t rs[32], rd[32];
@@ -256,36 +281,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(tDP + 32 * ch, rd);
         tmem_wait_ld();
         uint32_t pk[16], dk[16];
+        // P and dS of the chunk; the visibility test is compiled only into
+        // the copy that masked tiles run (predicating it into every tile
+        // costs a fifth of the kernel's time)
+        auto pds = [&](auto mk) {
+          constexpr bool kMasked = decltype(mk)::value;
 #pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
-          // log2 LSE and D of 4 query rows (broadcast shared-memory reads)
-          const float4 l4 = reinterpret_cast<const float4*>(lse_s + 32 * ch)[i4];
-          const float4 d4 = reinterpret_cast<const float4*>(dl_s + 32 * ch)[i4];
-          const float lz[4] = {l4.x, l4.y, l4.z, l4.w}, dz[4] = {d4.x, d4.y, d4.z, d4.w};
-          float pv[4], dsv[4];
+          for (int i4 = 0; i4 < 8; ++i4) {
+            // log2 LSE and D of 4 query rows (broadcast shared-memory reads,
+            // addressed in the shared window)
+            float4 l4, d4;
+            asm("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(l4.x), "=f"(l4.y), "=f"(l4.z), "=f"(l4.w)
+                : "r"(sL + 4u * (32 * ch + 4 * i4)));
+            asm("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(d4.x), "=f"(d4.y), "=f"(d4.z), "=f"(d4.w)
+                : "r"(sDl + 4u * (32 * ch + 4 * i4)));
+            const float lz[4] = {l4.x, l4.y, l4.z, l4.w}, dz[4] = {d4.x, d4.y, d4.z, d4.w};
+            float pv[4], dsv[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int qc = 32 * ch + 4 * i4 + e;  // query column in the tile
-            float pe = ex2_approx(fmaf(__uint_as_float(rs[4 * i4 + e]), p.c, -lz[e]));
-            if (masked) {
-              const int gi = q0 + qc + koff;  // diagonal key of query row q0 + qc
-              const bool vis = (q0 + qc < p.Nq) && (key < p.Nk) && (p.wl < 0 || key >= gi - p.wl) &&
-                               (p.wr < 0 || key <= gi + p.wr);
-              if (!vis) pe = 0.f;
+            for (int e = 0; e < 4; ++e) {
+              const int qc = 32 * ch + 4 * i4 + e;  // query column in the tile
+              float pe = ex2_approx(fmaf(__uint_as_float(rs[4 * i4 + e]), p.c, -lz[e]));
+              if constexpr (kMasked) {
+                const int gi = q0 + qc + koff;  // diagonal key of query row q0 + qc
+                const bool vis = (q0 + qc < p.Nq) && (key < p.Nk) && (p.wl < 0 || key >= gi - p.wl) &&
+                                 (p.wr < 0 || key <= gi + p.wr);
+                if (!vis) pe = 0.f;
+              }
+              pv[e] = pe;
+              dsv[e] = pe * (__uint_as_float(rd[4 * i4 + e]) - dz[e]);
             }
-            pv[e] = pe;
-            dsv[e] = pe * (__uint_as_float(rd[4 * i4 + e]) - dz[e]);
+            pk[2 * i4] = pack_bf16x2(pv[0], pv[1]);
+            pk[2 * i4 + 1] = pack_bf16x2(pv[2], pv[3]);
+            dk[2 * i4] = pack_bf16x2(dsv[0], dsv[1]);
+            dk[2 * i4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
           }
-          pk[2 * i4] = pack_bf16x2(pv[0], pv[1]);
-          pk[2 * i4 + 1] = pack_bf16x2(pv[2], pv[3]);
-          dk[2 * i4] = pack_bf16x2(dsv[0], dsv[1]);
-          dk[2 * i4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
-        }
+        };
+        if (masked)
+          pds(std::true_type{});
+        else
+          pds(std::false_type{});
         // bf16 P^T / dS^T over S^T / dP^T columns this warpgroup has consumed:
         // chunk ch goes to columns bf16_col(ch) (0, 16, 64, 80), so neither
         // warpgroup overwrites scores the other has yet to read
         tmem_st16(tS + bf16_col(ch), pk);
         tmem_st16(tDP + bf16_col(ch), dk);
+        // the dS buffer held the previous tile's dQ staging until both bulk
+        // reductions had read it
+        if (ch == 2 * wg && it > 0 &&
+            !mbar_wait_warp(bar(BB_STGREAD + 1), (it - 1) & 1, g, FA2_SITE_O_RESCALED, it)) {
+          ok = false;
+          break;
+        }
         // dS^T row into shared memory: queries [32 ch, 32 ch + 32) of key row
         // kr, MN-major SW128 (query chunk of 64 = 16 KiB block, 128 B per key)
 #pragma unroll
@@ -298,6 +344,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                        : "memory");
         }
       }
+      if (!ok) break;
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
@@ -309,9 +356,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         break;
       }
       tc_fence_after();
-      const int row = q0 + kr;
-      // Read the half row into registers and hand the columns back to the MMA
-      // at once; the atomics then overlap the next tile's products.
+      // Read the half row (query row q0 + kr) into registers and hand the
+      // columns back to the MMA at once; the reduction into the accumulator
+      // then overlaps the next tile's products.
       uint32_t r[D / 2];
 #pragma unroll
       for (int c = 0; c < D / 64; ++c)
@@ -319,14 +366,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(BB_DQFREE));
-      if (row < p.Nq) {
-        float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.Nq + row) * p.Hq + hq) * D + wg * (D / 2);
+      // Stage this half row (scaled) in the dS buffer -- free since the dQ MMA
+      // read it -- as D/64 boxes of 128 rows x 32 fp32 columns in the 128-byte
+      // swizzle of the dQ tensor map, then one thread adds the boxes into the
+      // fp32 accumulator with bulk (TMA) reductions.  The two warpgroups take
+      // turns on the buffer: warpgroup 1 stages once warpgroup 0's reductions
+      // have read it; the next tile's dS waits for warpgroup 1's.
+      if (wg == 1 && !mbar_wait_warp(bar(BB_STGREAD + 0), it & 1, g, FA2_SITE_O_RESCALED, it)) {
+        ok = false;
+        break;
+      }
+      {
+        const uint32_t sstg = sbase + C::kOffDS;
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i)
-          red_add_v4(dst + 4 * i, __uint_as_float(r[4 * i]) * p.scale, __uint_as_float(r[4 * i + 1]) * p.scale,
-                     __uint_as_float(r[4 * i + 2]) * p.scale, __uint_as_float(r[4 * i + 3]) * p.scale);
+        for (int bx = 0; bx < D / 64; ++bx)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t addr = sstg + bx * (kBlockM * 128) + kr * 128 + ((u ^ (kr & 7)) << 4);
+            const int c = 32 * bx + 4 * u;
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                         "f"(__uint_as_float(r[c]) * p.scale), "f"(__uint_as_float(r[c + 1]) * p.scale),
+                         "f"(__uint_as_float(r[c + 2]) * p.scale), "f"(__uint_as_float(r[c + 3]) * p.scale)
+                         : "memory");
+          }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(BB_STAGED + wg));
+        if (warp == 4 * wg && lane == 0) {
+          if (!mbar_wait(bar(BB_STAGED + wg), it & 1, g, FA2_SITE_O_RESCALED, it)) {
+            ok = false;
+          } else {
+#pragma unroll
+            for (int bx = 0; bx < D / 64; ++bx)
+              tma_reduce_add_4d(&tmDQ, sstg + bx * (kBlockM * 128), wg * (D / 2) + 32 * bx, hq, q0, b);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+            mbar_arrive(bar(BB_STGREAD + wg));
+          }
+        }
+        if (!__all_sync(0xffffffffu, ok)) break;
       }
     }
+    // the bulk reductions this thread issued are complete before the CTA exits
+    if (lane == 0 && (warp & 3) == 0) bulk_wait_group0();
     // ---- epilogue: WG0 writes dV, WG1 dK (scaled), rows of this key block ----
     if (ok && n_it > 0 && !mbar_wait_warp(bar(BB_DONE), 0, g, FA2_SITE_MMA_DRAIN, 0)) ok = false;
     tc_fence_after();
@@ -548,6 +629,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // ------------------------------- host side -------------------------------
 
+// 4-D map over the fp32 dQ accumulator [B, Nq, Hq, d] with a (32 x 1 x 128 x
+// 1) box and 128-byte swizzle: one box is 128 query rows x 32 columns of one
+// head, the unit of the bulk reductions.
+static bool encode_dq_acc(CUtensorMap* map, const float* base, int B, int N, int H, int d) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 4,
+                                 static_cast<cuuint64_t>(H) * d * 4,
+                                 static_cast<cuuint64_t>(N) * H * d * 4};
+  const cuuint32_t box[4] = {32, 1, static_cast<cuuint32_t>(kBlockM), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
 static int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                       const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
@@ -570,9 +669,10 @@ static int launch_bwd(const void* q, const void* k, const void* v, const void* o
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
       dq_acc, B, Hq, Nq);
   if (cudaGetLastError() != cudaSuccess) return FA2_ERR_LAUNCH;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   if (!encode_bnhd(&tq, q, B, Nq, Hq, D) || !encode_bnhd(&tk, k, B, Nk, Hkv, D) ||
-      !encode_bnhd(&tv, v, B, Nk, Hkv, D) || !encode_bnhd(&tdo, dout, B, Nq, Hq, D))
+      !encode_bnhd(&tv, v, B, Nk, Hkv, D) || !encode_bnhd(&tdo, dout, B, Nq, Hq, D) ||
+      !encode_dq_acc(&tdq, dq_acc, B, Nq, Hq, D))
     return FA2_ERR_LAUNCH;
   BwdParams p;
   p.lse2 = lse2;
@@ -591,7 +691,7 @@ static int launch_bwd(const void* q, const void* k, const void* v, const void* o
   p.c = scale * 1.4426950408889634f;
   p.limit_ns = 1000000000u;
   const dim3 grid(static_cast<unsigned>((Nk + kBlockN - 1) / kBlockN), Hkv, B);
-  fa2_bwd_kernel<D><<<grid, kBwdThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, p);
+  fa2_bwd_kernel<D><<<grid, kBwdThreads, C::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, p);
   if (cudaGetLastError() != cudaSuccess) return FA2_ERR_LAUNCH;
   const long long n4 = rows * D / 4;
   fa2_bwd_dq_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(

@@ -22,9 +22,12 @@
 // dV need no atomics (GQA sums the group's heads in place).  dQ is the only
 // output shared between CTAs: each CTA adds its 128 x d contribution per
 // query tile into an fp32 accumulator with TMA bulk reductions (the scaled
-// tile is staged in the shared-memory dS buffer once the dQ MMA has read it),
-// and a last kernel rounds the accumulator to bf16 (scale is applied before
-// the reduction).
+// tile is staged in the shared-memory slots of that tile's Q and dO, which
+// every MMA has finished reading once the dQ tile is complete), and a last
+// kernel rounds the accumulator to bf16 (scale is applied before the
+// reduction).  Each CTA walks its query tiles starting at a different one
+// (rotated by the key block), so the CTAs of one head running at the same
+// time add into different dQ rows.
 //
 // Per query tile (tensor memory: S^T | dP^T | dV | dK):
 //   MMA   S^T = K Q^T (SS), dP^T = V dO^T (SS)            -> "S ready"
@@ -35,9 +38,10 @@
 //         S^T columns, after the dV MMA read P^T: one thread's MMAs run in
 //         issue order)                                     -> "dQ ready"
 //   WG0/1 read dQ_tile, scale          -> "dQ free": the next tile's S^T
-//         may overwrite the columns; stage the half tile in the dS buffer
-//         and one thread per warpgroup issues its bulk reduce-add into the
-//         fp32 accumulator; the next tile's dS waits for that read.
+//         may overwrite the columns; WG0 stages its half in the tile's Q
+//         slot, WG1 in its dO slot, and one thread per warpgroup issues the
+//         bulk reduce-add into the fp32 accumulator; the producer refills a
+//         slot (two tiles later) once that reduction has read it.
 //
 // Roles: warps 0-3 (WG0) and 4-7 (WG1) split the query columns of P / dS
 // (one thread per key row) and of the dQ read-out (one thread per query
@@ -80,9 +84,9 @@ enum BwdBar {
   BB_DQ = 11,       // dQ tile complete
   BB_DQFREE = 12,   // dQ tile read out (128 WG1 threads)
   BB_DONE = 13,     // every MMA complete: dK, dV final
-  BB_STAGED = 14,   // [2] warpgroup wg's half of the dQ tile staged in the dS buffer (128 threads)
-  BB_STGREAD = 16,  // [2] warpgroup wg's bulk reduction has read the dS buffer (1 thread)
-  BB_COUNT = 18,
+  BB_STAGED = 14,   // [2] warpgroup wg's half of the dQ tile staged (128 threads)
+  BB_STGREAD = 16,  // [2 wg][2 slot] warpgroup wg's bulk reduction has read its staging slot (1 thread)
+  BB_COUNT = 20,
 };
 
 template <int D>
@@ -216,7 +220,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   int qt_lo, qt_hi;
   query_tiles_for(p, kb, qt_lo, qt_hi);
   const int n_qt = qt_hi - qt_lo + 1 > 0 ? qt_hi - qt_lo + 1 : 0;
-  const int n_it = n_qt * group;  // iteration it: head hk*group + it / n_qt, query tile qt_lo + it % n_qt
+  // iteration it: head hk*group + it / n_qt, query tile qt_lo + (it % n_qt + kb) % n_qt
+  const int n_it = n_qt * group;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -260,7 +265,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int it = 0; it < n_it && ok; ++it) {
       const int st = it & 1;
       const int hq = hk * group + it / n_qt;
-      const int q0 = (qt_lo + it % n_qt) * kBlockM;
+      const int q0 = (qt_lo + (it % n_qt + kb) % n_qt) * kBlockM;
       if (!mbar_wait_warp(bar(BB_SDP), it & 1, g, FA2_SITE_S_READY, it)) {
         ok = false;
         break;
@@ -325,13 +330,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // warpgroup overwrites scores the other has yet to read
         tmem_st16(tS + bf16_col(ch), pk);
         tmem_st16(tDP + bf16_col(ch), dk);
-        // the dS buffer held the previous tile's dQ staging until both bulk
-        // reductions had read it
-        if (ch == 2 * wg && it > 0 &&
-            !mbar_wait_warp(bar(BB_STGREAD + 1), (it - 1) & 1, g, FA2_SITE_O_RESCALED, it)) {
-          ok = false;
-          break;
-        }
         // dS^T row into shared memory: queries [32 ch, 32 ch + 32) of key row
         // kr, MN-major SW128 (query chunk of 64 = 16 KiB block, 128 B per key)
 #pragma unroll
@@ -366,18 +364,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(BB_DQFREE));
-      // Stage this half row (scaled) in the dS buffer -- free since the dQ MMA
-      // read it -- as D/64 boxes of 128 rows x 32 fp32 columns in the 128-byte
-      // swizzle of the dQ tensor map, then one thread adds the boxes into the
-      // fp32 accumulator with bulk (TMA) reductions.  The two warpgroups take
-      // turns on the buffer: warpgroup 1 stages once warpgroup 0's reductions
-      // have read it; the next tile's dS waits for warpgroup 1's.
-      if (wg == 1 && !mbar_wait_warp(bar(BB_STGREAD + 0), it & 1, g, FA2_SITE_O_RESCALED, it)) {
-        ok = false;
-        break;
-      }
+      // Stage this half row (scaled) as D/64 boxes of 128 rows x 32 fp32
+      // columns in the 128-byte swizzle of the dQ tensor map, then one thread
+      // adds the boxes into the fp32 accumulator with bulk (TMA) reductions.
+      // Warpgroup 0 stages in the tile's Q slot, warpgroup 1 in its dO slot
+      // (each is exactly one half at d = 64 and 128): every MMA that read them
+      // completed before the dQ tile did, and the producer loads tile it + 2
+      // into them only after the reductions have read them.
       {
-        const uint32_t sstg = sbase + C::kOffDS;
+        const uint32_t sstg = sbase + (wg == 0 ? C::kOffQ : C::kOffO) + (it & 1) * C::kTileBytes;
 #pragma unroll
         for (int bx = 0; bx < D / 64; ++bx)
 #pragma unroll
@@ -400,7 +395,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               tma_reduce_add_4d(&tmDQ, sstg + bx * (kBlockM * 128), wg * (D / 2) + 32 * bx, hq, q0, b);
             bulk_commit_group();
             bulk_wait_group_read0();
-            mbar_arrive(bar(BB_STGREAD + wg));
+            mbar_arrive(bar(BB_STGREAD + 2 * wg + (it & 1)));
           }
         }
         if (!__all_sync(0xffffffffu, ok)) break;
@@ -571,8 +566,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (; it < n_it && ok; ++it) {
       const int qs = it & 1, os = it % C::kOStages;
       const int hq = hk * group + it / n_qt;
-      const int q0 = (qt_lo + it % n_qt) * kBlockM;
-      if (it >= 2 && !mbar_wait_warp(bar(BB_QFREE + qs), ((it >> 1) - 1) & 1, g, FA2_SITE_KV_FREE, it)) {
+      const int q0 = (qt_lo + (it % n_qt + kb) % n_qt) * kBlockM;
+      if (it >= 2 && (!mbar_wait_warp(bar(BB_QFREE + qs), ((it >> 1) - 1) & 1, g, FA2_SITE_KV_FREE, it) ||
+                      !mbar_wait_warp(bar(BB_STGREAD + 0 + qs), ((it >> 1) - 1) & 1, g, FA2_SITE_KV_FREE, it))) {
         ok = false;
         break;
       }
@@ -595,7 +591,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       __syncwarp();
       if (it >= C::kOStages &&
-          !mbar_wait_warp(bar(BB_OFREE + os), ((it / C::kOStages) - 1) & 1, g, FA2_SITE_KV_FREE, it)) {
+          (!mbar_wait_warp(bar(BB_OFREE + os), ((it / C::kOStages) - 1) & 1, g, FA2_SITE_KV_FREE, it) ||
+           !mbar_wait_warp(bar(BB_STGREAD + 2 + os), ((it / C::kOStages) - 1) & 1, g, FA2_SITE_KV_FREE, it))) {
         ok = false;
         break;
       }

@@ -577,6 +577,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m_sc = 0.f;         // m_raw * c (0 while no key was visible)
       float l = 0.f;            // running denominator, relative to m_sc
       float lr = 0.f;           // bf16 rounding of each tile's largest probability, summed like l
+      // this row's visible keys [lo_abs, hi_abs]; tiles j >= j_hi cross some
+      // row's right bound or the key tail, tiles j < j_lo some row's left bound
+      // (ints: the host keeps Nq + Nk below 2^30 and each window below N)
+      const int hi_abs = (p.wr >= 0) ? min(row + koff + p.wr, p.Nk - 1) : p.Nk - 1;
+      const int lo_abs = (p.wl >= 0) ? row + koff - p.wl : 0;
+      const int j_hi = (((p.wr >= 0) ? min(r0t + koff + p.wr, p.Nk - 1) : p.Nk - 1) + 1) / kBlockN;
+      const int j_lo = (p.wl >= 0) ? (r0t + kBlockM - 1 + koff - p.wl + kBlockN - 1) / kBlockN : 0;
       for (int jj = 0; jj < ntt; ++jj) {
         const int j = pc.j0 + pc.jb + jj;  // K/V tile (absolute)
         if (!mbar_wait_warp(bar(BAR_S + t), s_cnt & 1, g, FA2_SITE_S_READY, j)) {
@@ -597,21 +604,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         // window edges (the causal diagonal) and the ragged key tail: only
         // tiles some row's bound falls into pay for masking
         const int kbase = j * kBlockN;
-        const bool masked = (kbase + kBlockN > p.Nk) ||
-                            (p.wr >= 0 && kbase + kBlockN - 1 > r0t + koff + p.wr) ||
-                            (p.wl >= 0 && kbase < r0t + kBlockM - 1 + koff - p.wl);
+        const bool masked = j >= j_hi || j < j_lo;
         if (masked) {
-          // visible columns [lo, hi] of this tile for this row (64-bit: the
-          // window bounds may lie far outside the tile)
-          const long long gk = static_cast<long long>(row) + koff - kbase;  // diagonal key, tile-relative
-          long long hi = min(kBlockN - 1, p.Nk - 1 - kbase);
-          if (p.wr >= 0 && gk + p.wr < hi) hi = gk + p.wr;
-          const long long lo = (p.wl >= 0) ? gk - p.wl : 0;
-          const int hi_i = static_cast<int>(hi < -1 ? -1 : hi);
-          const int lo_i = static_cast<int>(lo > kBlockN ? kBlockN : lo);
+          // visible columns [lo_i, hi_i] of this tile for this row
+          const int hi_i = max(min(hi_abs - kbase, kBlockN - 1), -1);
+          const int lo_i = min(lo_abs - kbase, kBlockN);
+          // one 32-bit visibility mask per 32 columns: a compact test, so the
+          // code unmasked tiles branch around stays small
 #pragma unroll
-          for (int i = 0; i < kBlockN; ++i)
-            if (i > hi_i || i < lo_i) s[i] = -INFINITY;
+          for (int k = 0; k < kBlockN / 32; ++k) {
+            const int lk = max(lo_i - 32 * k, 0), hk = min(hi_i - 32 * k, 31);
+            uint32_t vk = 0u;
+            if (hk >= lk) vk = (0xffffffffu >> (31 - hk)) & (0xffffffffu << lk);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (!((vk >> i) & 1u)) s[32 * k + i] = -INFINITY;
+          }
         }
         // row max: 8 independent chains of 3-input max (max is exact in any order)
         float mp[8];

@@ -7,6 +7,14 @@ to its own scale: max |err| <= 3e-2 * max |ref| and mean |err| <= 1e-2 *
 mean |ref|, with no NaN or Inf.  Where a gradient vanishes exactly (a row that
 sees one key has dS = P (dP - D) = 0) the GPU's dP - D is a rounding residue,
 so the scales have floors: 1e-3 for the max and 1e-4 for the mean.
+
+Row by row as well: every gradient row (one key's dK / dV, one query's dQ, d
+values) whose largest element is at least a tenth of the tensor's largest is
+held to its own scale, max |err_row| <= 1.5e-2 * max |ref_row| for dK and dV
+(each a sum of bf16 products with fp32 accumulation: a few units of 2^-9)
+and 3e-2 for dQ, whose dS = P (dP - D) loses relative precision where dP and
+D = dO . O (O rounded to bf16) nearly cancel.  Rows smaller than that are the
+ones whose gradient (nearly) vanishes; the tensor-wide bound covers them.
 """
 
 import numpy as np
@@ -19,6 +27,18 @@ from exact_tiled_attention_29_b200.inputs import Workload, bf16_bits, make_qkv
 pytestmark = pytest.mark.gpu
 
 MAX_REL, MEAN_REL = 3e-2, 1e-2
+ROW_REL = {"dQ": 3e-2, "dK": 1.5e-2, "dV": 1.5e-2}
+ROW_MIN = 0.1  # rows checked on their own scale: max |ref_row| >= ROW_MIN * max |ref|
+
+
+def check_rows(tag, name, a, r):
+    big = max(np.abs(r).max(), 1e-3)
+    err = np.abs(a - r).max(axis=-1)
+    rmax = np.abs(r).max(axis=-1)
+    sel = rmax >= ROW_MIN * big
+    if sel.any():
+        worst = (err[sel] / rmax[sel]).max()
+        assert worst <= ROW_REL[name], f"{tag} {name}: row-relative error {worst:.3g}"
 
 
 @pytest.fixture(scope="module")
@@ -52,6 +72,7 @@ def check(fa2, w, scale=None):
         assert err.max() <= MAX_REL * big, f"{w.name} {name}: max err {err.max():.3g} vs scale {big:.3g}"
         assert err.mean() <= MEAN_REL * max(np.abs(r).mean(), 1e-4), \
             f"{w.name} {name}: mean err {err.mean():.3g} vs mean {np.abs(r).mean():.3g}"
+        check_rows(w.name, name, a, r)
 
 
 @pytest.mark.parametrize("d", [64, 128])
@@ -97,3 +118,4 @@ def test_backward_local_window(fa2, window, d):
         big = max(np.abs(r).max(), 1e-3)
         assert err.max() <= MAX_REL * big, f"{window} {name}: max err {err.max():.3g} vs {big:.3g}"
         assert err.mean() <= MEAN_REL * max(np.abs(r).mean(), 1e-4), f"{window} {name}: mean err"
+        check_rows(str(window), name, a, r)

@@ -60,8 +60,9 @@ def parse_args():
                     help="fwd: the forward pass (the headline); bwd: fa2_backward on the forward's "
                          "outputs, FLOPs counted as 2.5x the forward's (five matrix products "
                          "instead of two)")
-    ap.add_argument("--schedule", default="units", choices=["units", "streamk"],
-                    help="streamk: fa2_forward_ws, one persistent block per SM over a workspace; "
+    ap.add_argument("--schedule", default="units", choices=["units", "streamk", "auto"],
+                    help="auto: fa2_forward_auto with a workspace (the library picks); "
+                         "streamk: fa2_forward_ws, one persistent block per SM over a workspace; "
                          "units: fa2_forward, one block per (query block, head, batch)")
     return ap.parse_args()
 
@@ -350,15 +351,17 @@ def run_fa2(args, w):
     # the library runs whole units on persistent CTAs when there are at least
     # two units per SM (the persistent instantiation of the kernel)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    persistent = args.schedule == "streamk" or fa2.fa2_launch_plan(
-        w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d)[1] >= 2 * sms
-    if args.schedule == "streamk" and w.windowed:
+    if args.schedule != "units" and w.windowed:
         raise SystemExit("the local-window workloads run the one-block-per-unit schedule only")
-    if args.schedule == "streamk":
+    # under "auto" the library's own choice decides which kernels a step runs
+    split = args.schedule == "streamk" or (
+        args.schedule == "auto" and
+        fa2.fa2_schedule_choice(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal, sms)[1] == 1)
+    persistent = split or fa2.fa2_launch_plan(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d)[1] >= 2 * sms
+    if args.schedule != "units":
         ws = fa2.alloc_workspace(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal, dev)
-        _, _, ctas, _ = fa2.fa2_streamk_plan(
-            w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
-            torch.cuda.get_device_properties(dev).multi_processor_count)
+    if split:
+        _, _, ctas, _ = fa2.fa2_streamk_plan(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal, sms)
         launches_per_step = 2 if ctas > 1 else 1
 
     def call(qq, kk, vv, oo, ll):
@@ -369,6 +372,9 @@ def run_fa2(args, w):
         elif ws is None:
             st = fa2.fa2_forward(qq, kk, vv, oo, ll, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
                                  w.softmax_scale, stream)
+        elif args.schedule == "auto":
+            st = fa2.fa2_forward_auto(qq, kk, vv, oo, ll, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d,
+                                      w.causal, w.softmax_scale, ws, ws.numel(), stream)
         else:
             st = fa2.fa2_forward_ws(qq, kk, vv, oo, ll, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d,
                                     w.causal, w.softmax_scale, ws, ws.numel(), stream)
@@ -440,6 +446,9 @@ def run_fa2(args, w):
             elif ws is None:
                 st = fa2.fa2_forward(qq, kk, vv, oo, ll, 1, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
                                      w.softmax_scale, stream)
+            elif args.schedule == "auto":
+                st = fa2.fa2_forward_auto(qq, kk, vv, oo, ll, 1, w.Hq, w.Hkv, w.Nq, w.Nk, w.d,
+                                          w.causal, w.softmax_scale, ws, ws.numel(), stream)
             else:
                 st = fa2.fa2_forward_ws(qq, kk, vv, oo, ll, 1, w.Hq, w.Hkv, w.Nq, w.Nk, w.d,
                                         w.causal, w.softmax_scale, ws, ws.numel(), stream)

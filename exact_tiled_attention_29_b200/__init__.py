@@ -9,7 +9,8 @@ does not load the library.
 _BINDING_NAMES = {
     "fa2_forward", "fa2_forward_local", "fa2_forward_ws", "fa2_backward", "fa2_backward_local",
     "fa2_backward_workspace_size", "attention_backward", "fa2_forward_static_ws", "fa2_workspace_size",
-    "fa2_streamk_plan", "fa2_persistent_plan", "FA2_STATIC_WS_BYTES",
+    "fa2_streamk_plan", "fa2_persistent_plan", "FA2_STATIC_WS_BYTES", "fa2_forward_auto",
+    "fa2_schedule_choice",
     "alloc_workspace", "fa2_status_string", "fa2_debug_status", "fa2_selftest_timeout",
     "fa2_num_blocks", "fa2_launch_plan", "attention", "FA2Error", "LIB_PATH", "FA2_OK",
     "STATUS_NAMES", "SITE_NAMES", "FA2_SITE_SELFTEST",

@@ -45,6 +45,8 @@ def _load() -> ctypes.CDLL:
     lib.fa2_forward.restype = ci
     lib.fa2_forward_ws.argtypes = [vp, vp, vp, vp, vp] + [ci] * 7 + [cf, vp, cll, vp]
     lib.fa2_forward_ws.restype = ci
+    lib.fa2_forward_auto.argtypes = [vp, vp, vp, vp, vp] + [ci] * 7 + [cf, vp, cll, vp]
+    lib.fa2_forward_auto.restype = ci
     lib.fa2_forward_local.argtypes = [vp, vp, vp, vp, vp] + [ci] * 8 + [cf, vp]
     lib.fa2_forward_local.restype = ci
     lib.fa2_forward_static_ws.argtypes = [vp, vp, vp, vp, vp] + [ci] * 7 + [cf, vp]
@@ -73,6 +75,8 @@ def _load() -> ctypes.CDLL:
     lib.fa2_streamk_plan.restype = ci
     lib.fa2_persistent_plan.argtypes = [ci] * 8 + [ip, ip, ci]
     lib.fa2_persistent_plan.restype = ci
+    lib.fa2_schedule_choice.argtypes = [ci] * 8 + [ip, llp, llp]
+    lib.fa2_schedule_choice.restype = ci
     return lib
 
 
@@ -122,6 +126,15 @@ def fa2_forward_ws(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale
                                    _stream(stream)))
 
 
+def fa2_forward_auto(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, workspace,
+                     workspace_bytes, stream) -> int:
+    """Whole units or stream-K, as the library's cost model picks (workspace may be None)."""
+    return int(_lib.fa2_forward_auto(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(Hq),
+                                     int(Hkv), int(Nq), int(Nk), int(d), int(bool(causal)),
+                                     float(softmax_scale), _ptr(workspace), int(workspace_bytes),
+                                     _stream(stream)))
+
+
 def fa2_forward_static_ws(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale,
                           stream) -> int:
     """Stream-K with the library's fixed scratch array; calls must not overlap."""
@@ -166,6 +179,15 @@ def fa2_streamk_plan(B, Hq, Hkv, Nq, Nk, d, causal, num_sms):
                                int(bool(causal)), int(num_sms), ctypes.byref(t), ctypes.byref(g),
                                ctypes.byref(w))
     return int(st), t.value, g.value, w.value
+
+
+def fa2_schedule_choice(B, Hq, Hkv, Nq, Nk, d, causal, num_sms):
+    """(status, split, cost_units, cost_split): fa2_forward_auto's choice."""
+    sp, cu, cs = ctypes.c_int(0), ctypes.c_longlong(0), ctypes.c_longlong(0)
+    st = _lib.fa2_schedule_choice(int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
+                                  int(bool(causal)), int(num_sms), ctypes.byref(sp), ctypes.byref(cu),
+                                  ctypes.byref(cs))
+    return int(st), sp.value, cu.value, cs.value
 
 
 def fa2_persistent_plan(B, Hq, Hkv, Nq, Nk, d, causal, num_sms, capacity=1 << 14):
@@ -219,14 +241,16 @@ def alloc_workspace(B, Hq, Hkv, Nq, Nk, d, causal, device):
 
 
 def attention(q, k, v, causal: bool = False, softmax_scale: float | None = None, out=None,
-              lse=None, stream=None, workspace=None, window=None):
+              lse=None, stream=None, workspace=None, window=None, schedule: str = "streamk"):
     """O, LSE for bf16 CUDA tensors q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d] (contiguous).
 
     Outputs are allocated with torch unless given; the work is one call to
-    ``fa2_forward`` on ``stream`` (default: torch's current stream), or to
-    ``fa2_forward_ws`` (stream-K schedule) when ``workspace`` -- a CUDA tensor
-    from ``alloc_workspace`` -- is given, or to ``fa2_forward_local`` when
-    ``window`` = (left, right) is given (causal then narrows the right side to 0).
+    ``fa2_forward`` on ``stream`` (default: torch's current stream), or, when
+    ``workspace`` -- a CUDA tensor from ``alloc_workspace`` -- is given, to
+    ``fa2_forward_ws`` (stream-K schedule; ``schedule="streamk"``) or
+    ``fa2_forward_auto`` (the library picks; ``schedule="auto"``), or to
+    ``fa2_forward_local`` when ``window`` = (left, right) is given (causal then
+    narrows the right side to 0).
     """
     import torch
 
@@ -257,10 +281,16 @@ def attention(q, k, v, causal: bool = False, softmax_scale: float | None = None,
     elif workspace is None:
         st = fa2_forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale, stream)
         where = "fa2_forward"
-    else:
+    elif schedule == "auto":
+        st = fa2_forward_auto(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale,
+                              workspace, workspace.numel() * workspace.element_size(), stream)
+        where = "fa2_forward_auto"
+    elif schedule == "streamk":
         st = fa2_forward_ws(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, causal, softmax_scale,
                             workspace, workspace.numel() * workspace.element_size(), stream)
         where = "fa2_forward_ws"
+    else:
+        raise ValueError(f"schedule must be 'streamk' or 'auto', not {schedule!r}")
     if st != FA2_OK:
         raise FA2Error(st, where)
     return out, lse

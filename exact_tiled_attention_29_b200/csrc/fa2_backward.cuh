@@ -39,14 +39,17 @@
 //         issue order)                                     -> "dQ ready"
 //   WG0/1 read dQ_tile, scale          -> "dQ free": the next tile's S^T
 //         may overwrite the columns; WG0 stages its half in the tile's Q
-//         slot, WG1 in its dO slot, and one thread per warpgroup issues the
-//         bulk reduce-add into the fp32 accumulator; the producer refills a
-//         slot (two tiles later) once that reduction has read it.
+//         slot, WG1 in its dO slot                   -> "half staged"
+//   RED   warp 10 (WG0's half) / 11 (WG1's) issues the bulk reduce-add into
+//         the fp32 accumulator and waits until it has read the slot -> "slot
+//         read"; the producer refills the slot (two tiles later) after that.
 //
 // Roles: warps 0-3 (WG0) and 4-7 (WG1) split the query columns of P / dS
 // (one thread per key row) and of the dQ read-out (one thread per query
-// row); warp 8 MMA issuer; warp 9 TMA producer; warps 10-11 idle.  No
-// register split: 384 threads leave 168 registers each.
+// row); warp 8 MMA issuer; warp 9 TMA producer; warps 10-11 dQ reducers (a
+// bulk async-group can only be waited for by the thread that issued it, so
+// the waits sit on warps with nothing else to do).  No register split: 384
+// threads leave 168 registers each.
 
 constexpr int kBwdThreads = 384;
 
@@ -84,9 +87,9 @@ enum BwdBar {
   BB_DQ = 11,       // dQ tile complete
   BB_DQFREE = 12,   // dQ tile read out (128 WG1 threads)
   BB_DONE = 13,     // every MMA complete: dK, dV final
-  BB_STAGED = 14,   // [2] warpgroup wg's half of the dQ tile staged (128 threads)
-  BB_STGREAD = 16,  // [2 wg][2 slot] warpgroup wg's bulk reduction has read its staging slot (1 thread)
-  BB_COUNT = 20,
+  BB_STAGED = 14,   // [2 wg][2 slot] warpgroup wg's half of the dQ tile staged (128 threads)
+  BB_STGREAD = 18,  // [2 wg][2 slot] the bulk reduction of that half has read the slot (1 thread)
+  BB_COUNT = 22,
 };
 
 template <int D>
@@ -229,7 +232,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       uint32_t cnt = 1;
       if (i == BB_QFULL || i == BB_QFULL + 1) cnt = 32;
       if (i == BB_PDS || i == BB_DQFREE) cnt = 2 * kBlockM;
-      if (i == BB_STAGED || i == BB_STAGED + 1) cnt = kBlockM;
+      if (i >= BB_STAGED && i < BB_STAGED + 4) cnt = kBlockM;
       mbar_init(bar(i), cnt);
     }
     fence_mbar_init();
@@ -365,7 +368,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(BB_DQFREE));
       // Stage this half row (scaled) as D/64 boxes of 128 rows x 32 fp32
-      // columns in the 128-byte swizzle of the dQ tensor map, then one thread
+      // columns in the 128-byte swizzle of the dQ tensor map; a reducer warp
       // adds the boxes into the fp32 accumulator with bulk (TMA) reductions.
       // Warpgroup 0 stages in the tile's Q slot, warpgroup 1 in its dO slot
       // (each is exactly one half at d = 64 and 128): every MMA that read them
@@ -385,24 +388,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                          : "memory");
           }
         fence_proxy_async_smem();
-        mbar_arrive(bar(BB_STAGED + wg));
-        if (warp == 4 * wg && lane == 0) {
-          if (!mbar_wait(bar(BB_STAGED + wg), it & 1, g, FA2_SITE_O_RESCALED, it)) {
-            ok = false;
-          } else {
-#pragma unroll
-            for (int bx = 0; bx < D / 64; ++bx)
-              tma_reduce_add_4d(&tmDQ, sstg + bx * (kBlockM * 128), wg * (D / 2) + 32 * bx, hq, q0, b);
-            bulk_commit_group();
-            bulk_wait_group_read0();
-            mbar_arrive(bar(BB_STGREAD + 2 * wg + (it & 1)));
-          }
-        }
-        if (!__all_sync(0xffffffffu, ok)) break;
+        mbar_arrive(bar(BB_STAGED + 2 * wg + (it & 1)));
       }
     }
-    // the bulk reductions this thread issued are complete before the CTA exits
-    if (lane == 0 && (warp & 3) == 0) bulk_wait_group0();
     // ---- epilogue: WG0 writes dV, WG1 dK (scaled), rows of this key block ----
     if (ok && n_it > 0 && !mbar_wait_warp(bar(BB_DONE), 0, g, FA2_SITE_MMA_DRAIN, 0)) ok = false;
     tc_fence_after();
@@ -614,6 +602,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_wait_warp(bar(BB_OFULL + j % C::kOStages), (j / C::kOStages) & 1, drain, FA2_SITE_LOAD_DRAIN, j);
       }
     }
+  } else if (warp >= 10) {
+    // ============ dQ reducers: warp 10 adds warpgroup 0's half, warp 11 warpgroup 1's ============
+    const int wg = warp - 10;
+    if (lane == 0) {
+      for (int it = 0; it < n_it; ++it) {
+        const int hq = hk * group + it / n_qt;
+        const int q0 = (qt_lo + (it % n_qt + kb) % n_qt) * kBlockM;
+        const uint32_t sstg = sbase + (wg == 0 ? C::kOffQ : C::kOffO) + (it & 1) * C::kTileBytes;
+        if (!mbar_wait(bar(BB_STAGED + 2 * wg + (it & 1)), (it >> 1) & 1, g, FA2_SITE_O_RESCALED, it)) break;
+#pragma unroll
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_reduce_add_4d(&tmDQ, sstg + bx * (kBlockM * 128), wg * (D / 2) + 32 * bx, hq, q0, b);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+        mbar_arrive(bar(BB_STGREAD + 2 * wg + (it & 1)));
+      }
+      // every reduction complete before the CTA exits
+      bulk_wait_group0();
+    }
+    __syncwarp();
   }
 
   tc_fence_before();

@@ -124,11 +124,16 @@ struct UnitTable {
 };
 struct NoTable {};
 
-// Range boundaries of a stream-K launch that are the first cut of a split
-// unit: the combine kernel runs one block row per entry.
+// The split units of a stream-K launch, one entry per unit, as the host
+// found them from the range boundaries: the partial buffer of its first piece
+// (slot = first cut - 1; piece q is in slot + q), its number of pieces, and
+// its coordinates.  The combine kernel runs one block row per entry.
 struct CutList {
   int n;
-  uint16_t c[kMaxTableCtas];
+  uint16_t slot[kMaxTableCtas];
+  uint16_t np[kMaxTableCtas];
+  uint16_t qb[kMaxTableCtas];
+  int bh[kMaxTableCtas];  // b * Hq + hq
 };
 
 // Warps 14-15 (otherwise idle) write the rows of units with no visible key.
@@ -1135,19 +1140,8 @@ template <int D>
 __global__ void __launch_bounds__(kCombineThreads)
     fa2_combine_kernel(const Params p, const __grid_constant__ CutList cuts) {
   using C = Cfg<D>;
-  const int c = cuts.c[blockIdx.x];
-  const int bc = range_start(p.span, p.rem, p.G, c);
-  PieceIter<true> it;
-  it.HB = p.B * p.Hq;
-  it.seek_round(p, bc);
-  const int w = PieceIter<true>::cost(it.n);
-  const int k = (bc - it.cum) / w;
-  const int s0 = it.cum + k * w + kUnitCost;  // position of the unit's iteration 0
-  if (!(bc > s0 && bc <= s0 + it.n - 1)) return;                  // B_c cuts no unit
-  if (c > 1 && range_start(p.span, p.rem, p.G, c - 1) > s0) return;  // not the unit's first cut
-  const int np = first_boundary_above(p, s0 + it.n - 1) - c + 1;   // pieces of the unit
-  const int slot = c - 1;                                          // CTA of piece 0
-  const int qb = p.n_qblk - 1 - it.r, b = k / p.Hq, hq = k % p.Hq;
+  const int slot = cuts.slot[blockIdx.x], np = cuts.np[blockIdx.x], qb = cuts.qb[blockIdx.x];
+  const int b = cuts.bh[blockIdx.x] / p.Hq, hq = cuts.bh[blockIdx.x] % p.Hq;
 
   const int rr = static_cast<int>(blockIdx.y) * kCombineRows + static_cast<int>(threadIdx.x) / 4;
   const int f4 = threadIdx.x % 4;
@@ -1160,8 +1154,9 @@ __global__ void __launch_bounds__(kCombineThreads)
   };
   // One pass over the pieces in batches of kBatch, every load of a batch in
   // flight at once (statistics and O together); the accumulator follows the
-  // running max across batches.  A unit has at most a few tens of pieces, so
-  // this is one or two round trips to memory per thread.
+  // running max across batches.  A unit is cut into about G / units pieces,
+  // so this is one or two round trips to memory per thread.  (Batches of 16
+  // take 154 registers, one block per SM, and measured no faster.)
   constexpr int kBatch = 8;
   float m_run = -INFINITY, l_tot = 0.f, lr_tot = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1323,6 +1318,55 @@ static Plan make_plan(int B, int Hq, int Nq, int Nk, Window win, int d, int num_
   return pl;
 }
 
+// Which schedule a call with a workspace should take.  Both are priced in
+// K/V-tile iterations of one CTA, a unit costing its tiles + kUnitCost:
+// whole units finish when the busiest SM does (longest-first list
+// scheduling of the units, one per CTA); split-KV spreads the summed cost
+// evenly over G CTAs and adds the merge.  A split-KV iteration measured
+// 1.25-1.35x slower than a whole-unit one (partial outputs, the merge, short
+// pieces), so split-KV is taken only when it predicts a clear win, and only
+// with fewer units than two per SM (the persistent whole-unit schedule
+// balances anything larger to within a few percent) ("FlashAttention-2 and
+// -3: From Algebra to GPU Scheduling", "Another use of mergeable statistics":
+// splitting keys buys parallelism when the queries alone give too little).
+constexpr double kSplitMargin = 1.5;
+constexpr int kMergeCost = 4;
+struct ScheduleChoice {
+  int split = 0;
+  long long mk_units = 0, mk_split = 0;
+};
+
+static ScheduleChoice choose_schedule(int B, int Hq, int Nq, int Nk, Window win, int d, int sms) {
+  ScheduleChoice ch;
+  const Plan pl = make_plan(B, Hq, Nq, Nk, win, d, sms);
+  if (pl.G <= 0 || sms <= 0) return ch;
+  const long long HB = static_cast<long long>(B) * Hq;
+  long long units_ne = 0;
+  for (int qb = 0; qb < pl.n_qblk; ++qb)
+    if (unit_tiles(Nq, Nk, win, qb) > 0) units_ne += HB;
+  ch.mk_split = (pl.T + pl.G - 1) / pl.G + kMergeCost;
+  if (units_ne >= 2LL * sms) {  // balanced persistent plan: about the average
+    ch.mk_units = (pl.T + sms - 1) / sms;
+    return ch;
+  }
+  std::vector<long long> cost;
+  for (int qb = pl.n_qblk - 1; qb >= 0; --qb) {
+    const int n = unit_tiles(Nq, Nk, win, qb);
+    if (n > 0) cost.insert(cost.end(), static_cast<size_t>(HB), n + kUnitCost);
+  }
+  std::sort(cost.begin(), cost.end(), std::greater<long long>());
+  std::priority_queue<long long, std::vector<long long>, std::greater<long long>> load;
+  for (int i = 0; i < sms; ++i) load.push(0);
+  for (long long c : cost) {
+    const long long l = load.top() + c;
+    load.pop();
+    load.push(l);
+    ch.mk_units = std::max(ch.mk_units, l);
+  }
+  ch.split = (kSplitMargin * static_cast<double>(ch.mk_split) < static_cast<double>(ch.mk_units)) ? 1 : 0;
+  return ch;
+}
+
 // Plan of persistent whole units (UnitTable).  The heavier units are listed in
 // groups of consecutive (batch, head) pairs -- whole GQA groups, about one
 // wave of units per group -- heaviest first inside each group; the light
@@ -1399,10 +1443,18 @@ static bool first_cuts(const Params& p, Window win, CutList& cuts) {
     }
     const long long w = cost(n);
     const long long k = (bc - cum) / w;
-    const long long s0 = cum + k * w + kUnitCost;
+    const long long s0 = cum + k * w + kUnitCost;  // position of the unit's iteration 0
     const bool cuts_unit = bc > s0 && bc <= s0 + n - 1;
     const bool first = c == 1 || range_start(p.span, p.rem, p.G, c - 1) <= s0;
-    if (cuts_unit && first) cuts.c[cuts.n++] = static_cast<uint16_t>(c);
+    if (!cuts_unit || !first) continue;
+    // pieces: one per range that overlaps the unit's iterations [s0, s0 + n)
+    int c_end = c;
+    while (c_end + 1 < p.G && range_start(p.span, p.rem, p.G, c_end + 1) <= s0 + n - 1) ++c_end;
+    const int i = cuts.n++;
+    cuts.slot[i] = static_cast<uint16_t>(c - 1);
+    cuts.np[i] = static_cast<uint16_t>(c_end - c + 2);
+    cuts.qb[i] = static_cast<uint16_t>(p.n_qblk - 1 - r);
+    cuts.bh[i] = static_cast<int>(k);
   }
   return true;
 }
@@ -1602,6 +1654,30 @@ extern "C" int fa2_forward_ws(const void* q, const void* k, const void* v, void*
   if (!workspace) return FA2_ERR_NULL_POINTER;
   return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal_window(causal), softmax_scale,
                       workspace, workspace_bytes, stream);
+}
+
+extern "C" int fa2_schedule_choice(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, int num_sms,
+                                   int* split, long long* cost_units, long long* cost_split) {
+  const int sv = validate_shape(B, Hq, Hkv, Nq, Nk, d);
+  if (sv != FA2_OK) return sv;
+  if (num_sms <= 0) return FA2_ERR_BAD_SHAPE;
+  const ScheduleChoice ch = choose_schedule(B, Hq, Nq, Nk, causal_window(causal), d, num_sms);
+  if (split) *split = ch.split;
+  if (cost_units) *cost_units = ch.mk_units;
+  if (cost_split) *cost_split = ch.mk_split;
+  return FA2_OK;
+}
+
+extern "C" int fa2_forward_auto(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                                float softmax_scale, void* workspace, long long workspace_bytes,
+                                void* stream) {
+  const int sv = validate_shape(B, Hq, Hkv, Nq, Nk, d);
+  if (sv != FA2_OK) return sv;
+  const ScheduleChoice ch = choose_schedule(B, Hq, Nq, Nk, causal_window(causal), d, sm_count());
+  const bool split = ch.split && workspace;
+  return forward_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal_window(causal), softmax_scale,
+                      split ? workspace : nullptr, split ? workspace_bytes : 0, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -149,6 +149,34 @@ int fa2_forward_ws(const void* q, const void* k, const void* v, void* o, float* 
                    void* workspace, long long workspace_bytes, void* stream);
 
 /*
+ * fa2_forward_auto -- fa2_forward or fa2_forward_ws, whichever the library
+ * predicts to be faster for this problem on the current device.  Both
+ * schedules are priced in K/V-tile iterations of one block (a unit costs its
+ * tiles plus the fixed per-unit cost): whole units finish when the busiest SM
+ * does (longest-first list scheduling of the units, or the average when the
+ * units number at least two per SM and the persistent plan balances them);
+ * split-KV spreads the summed cost over one block per SM and adds the merge.
+ * Split-KV is taken only when there are fewer than two units per SM and its
+ * price times 1.5 is still below the whole-unit price (a split-KV iteration
+ * measured 1.25-1.35x dearer: partial outputs, the merge, short pieces) --
+ * a short query block against a long key sequence, where one block per unit
+ * would leave most SMs idle ("FlashAttention-2 and -3: From Algebra to GPU
+ * Scheduling", "Another use of mergeable statistics").
+ *
+ *   workspace        as in fa2_forward_ws, or NULL: then whole units always
+ *   workspace_bytes  its size (at least fa2_workspace_size(...) when split-KV
+ *                    is chosen)
+ *   (other arguments as in fa2_forward)
+ *
+ * Returns what the chosen entry point returns (FA2_ERR_WORKSPACE when
+ * split-KV is chosen and the workspace is too small).  The result equals
+ * either schedule's up to the order of floating-point rounding.
+ */
+int fa2_forward_auto(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                     int Hkv, int Nq, int Nk, int d, int causal, float softmax_scale,
+                     void* workspace, long long workspace_bytes, void* stream);
+
+/*
  * fa2_workspace_size -- bytes of workspace fa2_forward_ws needs for this
  * problem on the current device: two partials of 2 x 128 x (d + 3) floats per
  * SM (0 when the work fits one block).  Returns -1 for an invalid shape (as fa2_forward validates it),
@@ -331,6 +359,17 @@ int fa2_persistent_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causa
  */
 int fa2_streamk_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, int num_sms,
                      long long* total_iters, int* ctas, long long* workspace_bytes);
+
+/*
+ * fa2_schedule_choice: the choice fa2_forward_auto makes on a GPU with
+ * num_sms SMs -- *split = 1 for split-KV (fa2_forward_ws), 0 for whole units
+ * -- and the two prices it compares, in K/V-tile iterations of the busiest
+ * block (*cost_split includes the merge).  Any output pointer may be NULL.
+ * Returns an fa2_status_code (validation as in fa2_forward, minus pointers;
+ * FA2_ERR_BAD_SHAPE for num_sms <= 0).  No CUDA call.
+ */
+int fa2_schedule_choice(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, int num_sms,
+                        int* split, long long* cost_units, long long* cost_split);
 
 #ifdef __cplusplus
 }

@@ -267,3 +267,37 @@ def test_persistent_units_schedule(fa2, w):
     assert st == 0 and units >= 2 * torch.cuda.get_device_properties(0).multi_processor_count
     rows = sample_rows(w, 300, seed=74)
     check_case(fa2, w, rows=rows)
+
+
+# ---- fa2_forward_auto: the schedule the library picks ----
+
+@pytest.mark.parametrize("w", [
+    Workload("auto_shortq", 1, 4, 4, 256, 8192, 128, False, seed=41),   # split-KV
+    Workload("auto_units", 2, 8, 4, 2048, 2048, 64, True, seed=42),     # whole units
+    Workload("auto_long_unit", 1, 1, 1, 300, 20000, 64, True, seed=43),
+])
+def test_auto_equals_the_schedule_it_picks(fa2, w):
+    dev = torch.device("cuda")
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    st, split, cu, cs = fa2.fa2_schedule_choice(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal, sms)
+    assert st == 0
+    q, k, v = make_qkv(w)
+    picked = run_gpu(fa2, q, k, v, w.causal, w.softmax_scale, sched="streamk" if split else "units")
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    ws = fa2.alloc_workspace(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal, dev)
+    o, lse = fa2.attention(qd, kd, vd, causal=w.causal, workspace=ws, schedule="auto")
+    o0 = torch.empty_like(qd)
+    l0 = torch.empty_like(lse)
+    st = fa2.fa2_forward_auto(qd, kd, vd, o0, l0, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal,
+                              w.softmax_scale, None, 0, torch.cuda.current_stream())
+    assert st == 0
+    torch.cuda.synchronize()
+    assert fa2.fa2_debug_status(None) == 0
+    # bit for bit the schedule it picked; with no workspace, whole units
+    assert np.array_equal(o.float().cpu().numpy(), picked[0]) and np.array_equal(lse.cpu().numpy(), picked[1])
+    units = run_gpu(fa2, q, k, v, w.causal, w.softmax_scale, sched="units")
+    assert np.array_equal(o0.float().cpu().numpy(), units[0]) and np.array_equal(l0.cpu().numpy(), units[1])
+    if w.name == "auto_shortq":
+        assert split == 1
+    if w.name == "auto_units":
+        assert split == 0

@@ -21,11 +21,11 @@
 // tile of every query head of its group that sees any of its keys, so dK and
 // dV need no atomics (GQA sums the group's heads in place).  dQ is the only
 // output shared between CTAs: each CTA adds its 128 x d contribution per
-// query tile into an fp32 accumulator with TMA bulk reductions (the scaled
-// tile is staged in the shared-memory slots of that tile's Q and dO, which
-// every MMA has finished reading once the dQ tile is complete), and a last
-// kernel rounds the accumulator to bf16 (scale is applied before the
-// reduction).  Each CTA walks its query tiles starting at a different one
+// query tile into an fp32 accumulator -- half by vector reductions from
+// registers, half by a TMA bulk reduction staged in the shared-memory slot of
+// that tile's dO, which every MMA has finished reading once the dQ tile is
+// complete -- and a last kernel rounds the accumulator to bf16 (scale is
+// applied before the reduction).  Each CTA walks its query tiles starting at a different one
 // (rotated by the key block), so the CTAs of one head running at the same
 // time add into different dQ rows.
 //
@@ -38,18 +38,18 @@
 //         S^T columns, after the dV MMA read P^T: one thread's MMAs run in
 //         issue order)                                     -> "dQ ready"
 //   WG0/1 read dQ_tile, scale          -> "dQ free": the next tile's S^T
-//         may overwrite the columns; WG0 stages its half in the tile's Q
-//         slot, WG1 in its dO slot                   -> "half staged"
-//   RED   warp 10 (WG0's half) / 11 (WG1's) issues the bulk reduce-add into
-//         the fp32 accumulator and waits until it has read the slot -> "slot
-//         read"; the producer refills the slot (two tiles later) after that.
+//         may overwrite the columns; WG0 adds its half with red.global,
+//         WG1 stages its half in the tile's dO slot  -> "half staged"
+//   RED   warp 10 issues the bulk reduce-add of WG1's half and waits until
+//         it has read the slot -> "slot read"; the producer refills the slot
+//         (two tiles later) after that.
 //
 // Roles: warps 0-3 (WG0) and 4-7 (WG1) split the query columns of P / dS
 // (one thread per key row) and of the dQ read-out (one thread per query
-// row); warp 8 MMA issuer; warp 9 TMA producer; warps 10-11 dQ reducers (a
-// bulk async-group can only be waited for by the thread that issued it, so
-// the waits sit on warps with nothing else to do).  No register split: 384
-// threads leave 168 registers each.
+// row); warp 8 MMA issuer; warp 9 TMA producer; warp 10 dQ reducer (a bulk
+// async-group can only be waited for by the thread that issued it, so the
+// wait sits on a warp with nothing else to do); warp 11 idle.  No register
+// split: 384 threads leave 168 registers each.
 
 constexpr int kBwdThreads = 384;
 
@@ -75,6 +75,11 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
 __device__ __forceinline__ void bulk_wait_group0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
+// Element-wise fp32 add of four consecutive floats into global memory.
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
 
 enum BwdBar {
   BB_KV = 0,        // K and V tiles of this CTA landed (TMA tx)
@@ -87,9 +92,9 @@ enum BwdBar {
   BB_DQ = 11,       // dQ tile complete
   BB_DQFREE = 12,   // dQ tile read out (128 WG1 threads)
   BB_DONE = 13,     // every MMA complete: dK, dV final
-  BB_STAGED = 14,   // [2 wg][2 slot] warpgroup wg's half of the dQ tile staged (128 threads)
-  BB_STGREAD = 18,  // [2 wg][2 slot] the bulk reduction of that half has read the slot (1 thread)
-  BB_COUNT = 22,
+  BB_STAGED = 14,   // [2 slot] warpgroup 1's half of the dQ tile staged in the dO slot (128 threads)
+  BB_STGREAD = 16,  // [2 slot] its bulk reduction has read the slot (1 thread)
+  BB_COUNT = 18,
 };
 
 template <int D>
@@ -232,7 +237,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       uint32_t cnt = 1;
       if (i == BB_QFULL || i == BB_QFULL + 1) cnt = 32;
       if (i == BB_PDS || i == BB_DQFREE) cnt = 2 * kBlockM;
-      if (i >= BB_STAGED && i < BB_STAGED + 4) cnt = kBlockM;
+      if (i == BB_STAGED || i == BB_STAGED + 1) cnt = kBlockM;
       mbar_init(bar(i), cnt);
     }
     fence_mbar_init();
@@ -367,15 +372,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(BB_DQFREE));
-      // Stage this half row (scaled) as D/64 boxes of 128 rows x 32 fp32
-      // columns in the 128-byte swizzle of the dQ tensor map; a reducer warp
-      // adds the boxes into the fp32 accumulator with bulk (TMA) reductions.
-      // Warpgroup 0 stages in the tile's Q slot, warpgroup 1 in its dO slot
-      // (each is exactly one half at d = 64 and 128): every MMA that read them
-      // completed before the dQ tile did, and the producer loads tile it + 2
-      // into them only after the reductions have read them.
-      {
-        const uint32_t sstg = sbase + (wg == 0 ? C::kOffQ : C::kOffO) + (it & 1) * C::kTileBytes;
+      // Add this half row (scaled) into the fp32 accumulator.  The TMA unit
+      // also brings in every tile's Q and dO, so the two halves take
+      // different paths: warpgroup 0 uses vector reductions from registers
+      // (the load/store path), warpgroup 1 a bulk (TMA) reduction.
+      if (wg == 0) {
+        const int row = q0 + kr;
+        if (row < p.Nq) {
+          float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.Nq + row) * p.Hq + hq) * D;
+#pragma unroll
+          for (int i = 0; i < D / 8; ++i)
+            red_add_v4(dst + 4 * i, __uint_as_float(r[4 * i]) * p.scale, __uint_as_float(r[4 * i + 1]) * p.scale,
+                       __uint_as_float(r[4 * i + 2]) * p.scale, __uint_as_float(r[4 * i + 3]) * p.scale);
+        }
+      } else {
+        // staged as D/64 boxes of 128 rows x 32 fp32 columns in the 128-byte
+        // swizzle of the dQ tensor map, in the tile's dO slot (exactly one
+        // half tile at d = 64 and 128): every MMA that read it completed
+        // before the dQ tile did, and the producer loads tile it + 2 into it
+        // only after the reduction has read it
+        const uint32_t sstg = sbase + C::kOffO + (it & 1) * C::kTileBytes;
 #pragma unroll
         for (int bx = 0; bx < D / 64; ++bx)
 #pragma unroll
@@ -388,7 +404,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                          : "memory");
           }
         fence_proxy_async_smem();
-        mbar_arrive(bar(BB_STAGED + 2 * wg + (it & 1)));
+        mbar_arrive(bar(BB_STAGED + (it & 1)));
       }
     }
     // ---- epilogue: WG0 writes dV, WG1 dK (scaled), rows of this key block ----
@@ -555,8 +571,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int qs = it & 1, os = it % C::kOStages;
       const int hq = hk * group + it / n_qt;
       const int q0 = (qt_lo + (it % n_qt + kb) % n_qt) * kBlockM;
-      if (it >= 2 && (!mbar_wait_warp(bar(BB_QFREE + qs), ((it >> 1) - 1) & 1, g, FA2_SITE_KV_FREE, it) ||
-                      !mbar_wait_warp(bar(BB_STGREAD + 0 + qs), ((it >> 1) - 1) & 1, g, FA2_SITE_KV_FREE, it))) {
+      if (it >= 2 && !mbar_wait_warp(bar(BB_QFREE + qs), ((it >> 1) - 1) & 1, g, FA2_SITE_KV_FREE, it)) {
         ok = false;
         break;
       }
@@ -580,7 +595,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       __syncwarp();
       if (it >= C::kOStages &&
           (!mbar_wait_warp(bar(BB_OFREE + os), ((it / C::kOStages) - 1) & 1, g, FA2_SITE_KV_FREE, it) ||
-           !mbar_wait_warp(bar(BB_STGREAD + 2 + os), ((it / C::kOStages) - 1) & 1, g, FA2_SITE_KV_FREE, it))) {
+           !mbar_wait_warp(bar(BB_STGREAD + os), ((it / C::kOStages) - 1) & 1, g, FA2_SITE_KV_FREE, it))) {
         ok = false;
         break;
       }
@@ -602,21 +617,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_wait_warp(bar(BB_OFULL + j % C::kOStages), (j / C::kOStages) & 1, drain, FA2_SITE_LOAD_DRAIN, j);
       }
     }
-  } else if (warp >= 10) {
-    // ============ dQ reducers: warp 10 adds warpgroup 0's half, warp 11 warpgroup 1's ============
-    const int wg = warp - 10;
+  } else if (warp == 10) {
+    // ============ dQ reducer: warpgroup 1's staged half, one bulk reduction per tile ============
     if (lane == 0) {
       for (int it = 0; it < n_it; ++it) {
         const int hq = hk * group + it / n_qt;
         const int q0 = (qt_lo + (it % n_qt + kb) % n_qt) * kBlockM;
-        const uint32_t sstg = sbase + (wg == 0 ? C::kOffQ : C::kOffO) + (it & 1) * C::kTileBytes;
-        if (!mbar_wait(bar(BB_STAGED + 2 * wg + (it & 1)), (it >> 1) & 1, g, FA2_SITE_O_RESCALED, it)) break;
+        const uint32_t sstg = sbase + C::kOffO + (it & 1) * C::kTileBytes;
+        if (!mbar_wait(bar(BB_STAGED + (it & 1)), (it >> 1) & 1, g, FA2_SITE_O_RESCALED, it)) break;
 #pragma unroll
         for (int bx = 0; bx < D / 64; ++bx)
-          tma_reduce_add_4d(&tmDQ, sstg + bx * (kBlockM * 128), wg * (D / 2) + 32 * bx, hq, q0, b);
+          tma_reduce_add_4d(&tmDQ, sstg + bx * (kBlockM * 128), D / 2 + 32 * bx, hq, q0, b);
         bulk_commit_group();
         bulk_wait_group_read0();
-        mbar_arrive(bar(BB_STGREAD + 2 * wg + (it & 1)));
+        mbar_arrive(bar(BB_STGREAD + (it & 1)));
       }
       // every reduction complete before the CTA exits
       bulk_wait_group0();

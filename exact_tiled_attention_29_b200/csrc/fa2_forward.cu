@@ -118,9 +118,15 @@ constexpr float kRescaleThreshold = 8.f;
 // deal units round robin instead.
 constexpr int kMaxTableCtas = 160;
 constexpr int kMaxTableUnits = 8192;
+// An entry is a unit index u = round * B * Hq + (b * Hq + hq), or -- with
+// kHalfTile0 / kHalfTile1 added -- only that unit's first or second 128-row
+// query tile (a half unit: the two halves of a unit may run on two CTAs).
+constexpr int kUnitBits = 13;
+constexpr int kHalfTile0 = 1 << kUnitBits, kHalfTile1 = 2 << kUnitBits;
+static_assert(kMaxTableUnits <= (1 << kUnitBits), "unit index bits");
 struct UnitTable {
   uint16_t start[kMaxTableCtas + 1];  // CTA c runs unit[start[c] .. start[c+1]) in that order
-  uint16_t unit[kMaxTableUnits];      // unit index u = round * B * Hq + (b * Hq + hq)
+  uint16_t unit[kMaxTableUnits];      // entries as above
 };
 struct NoTable {};
 
@@ -274,6 +280,7 @@ struct Piece {
   int jb, je;       // K/V tiles [jb, je) of the unit
   int nt0, nt1;     // K/V tiles of Q0 / Q1 over the whole unit
   int a0, a1;       // iterations of Q0 / Q1 in this piece
+  int own;          // query tiles whose outputs this piece writes (bit t; a half unit owns one)
   int split;        // the unit is shared with other pieces
   int slot;         // CTA that runs the unit's first piece (the partial buffers count from it)
   int npieces;      // pieces of the unit
@@ -322,6 +329,7 @@ struct PieceIter {
     pc.nt1 = u.n1;
     pc.a0 = max(0, min(je, pc.nt0) - jb);
     pc.a1 = max(0, min(je, pc.nt1) - jb);
+    pc.own = 3;
   }
 
   // (batch, head, query block) of the current piece, recomputed from the
@@ -414,11 +422,12 @@ struct PieceIter {
       // when w is odd) so each CTA's heavy and light units pair up.
       const int u_count = p.r_empty * HB;  // units with some visible key
       const int c = static_cast<int>(blockIdx.x);
-      int u;
+      int u, half = 0;
       if (p.tab) {
         const int i = plan->start[c] + x;
         if (i >= plan->start[c + 1]) return false;
-        u = plan->unit[i];
+        u = plan->unit[i] & ((1 << kUnitBits) - 1);
+        half = plan->unit[i] >> kUnitBits;
       } else {
         u = x * p.G + ((x & 1) ? p.G - 1 - c : c);
       }
@@ -429,6 +438,17 @@ struct PieceIter {
       cum = 0;
       n = unit_tiles(p.Nq, p.Nk, window_of(p), p.n_qblk - 1 - r);
       fill(p, pc, r, k_cur, 0, n);
+      // a half unit walks only its query tile's prefix of the unit's K/V
+      // range (every K/V item the piece loads must be used, which frees it)
+      if (half == 1) {  // first query tile only: the second is another CTA's
+        pc.a1 = 0;
+        pc.je = pc.jb + pc.a0;
+        pc.own = 1;
+      } else if (half == 2) {
+        pc.a0 = 0;
+        pc.je = pc.jb + pc.a1;
+        pc.own = 2;
+      }
       return true;
     }
     if (state) {  // the head piece: iterations [0, B_{c+1} - position of iteration 0)
@@ -812,7 +832,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(BAR_FCONS + t));
         tc_fence_after();
         const uint32_t tO = tmem + lane_off + C::col_o(t);
-        if (!pc.split) {
+        if (!((pc.own >> t) & 1)) {
+          // the other half of a split-in-two unit writes this query tile
+        } else if (!pc.split) {
           // single division per row, bf16 O, LSE = ln(sum exp(scale * s))
           const int row = pc.qb * kRowsPerCta + t * kBlockM + rt;
           const bool valid = row < p.Nq;
@@ -1399,21 +1421,44 @@ static bool plan_units(int B, int Hq, int Hkv, int Nq, int Nk, Window win, int n
   for (int r = 0; r < r_empty; ++r) (5 * cost[r] > 2 * cmax ? heavy : light).push_back(r);
   std::stable_sort(light.begin(), light.end(), [&](int a, int b) { return cost[a] > cost[b]; });
   // list scheduling: the next unit goes to the CTA with the least planned work
+  // the list of units in dealing order
+  std::vector<std::pair<int, long long>> order;  // (round, b * Hq + hq)
+  for (long long k0 = 0; k0 < HB; k0 += hg)
+    for (int r : heavy)
+      for (long long k = k0; k < std::min(HB, k0 + hg); ++k) order.push_back({r, k});
+  for (int r : light)
+    for (long long k = 0; k < HB; ++k) order.push_back({r, k});
+  // Units that would make a last, at most half-full wave are dealt as two
+  // single-tile halves each, so twice as many CTAs share that wave: with R
+  // units left after the full waves (2 R <= G), the slowest CTA finishes one
+  // half unit after the full waves instead of one whole unit.  A half costs
+  // its tiles x 5/8 + the fixed cost (one query tile's softmax and MMAs per
+  // K/V tile, the K/V stream unchanged).
+  const long long rest = units % G;
+  long long n_half = (2 * rest <= G && units + rest <= kMaxTableUnits) ? rest : 0;
   using Slot = std::pair<long long, int>;  // (planned work, CTA)
   std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> free_at;
   for (int c = 0; c < G; ++c) free_at.push({0, c});
   std::vector<std::vector<uint16_t>> lists(G);
-  auto assign = [&](int r, long long k) {
+  auto assign = [&](int entry, int c_work) {
     const Slot sl = free_at.top();
     free_at.pop();
-    lists[sl.second].push_back(static_cast<uint16_t>(r * HB + k));
-    free_at.push({sl.first + cost[r], sl.second});
+    lists[sl.second].push_back(static_cast<uint16_t>(entry));
+    free_at.push({sl.first + c_work, sl.second});
   };
-  for (long long k0 = 0; k0 < HB; k0 += hg)
-    for (int r : heavy)
-      for (long long k = k0; k < std::min(HB, k0 + hg); ++k) assign(r, k);
-  for (int r : light)
-    for (long long k = 0; k < HB; ++k) assign(r, k);
+  const long long first_half = static_cast<long long>(order.size()) - n_half;
+  for (long long i = 0; i < static_cast<long long>(order.size()); ++i) {
+    const int r = order[i].first;
+    const int u = static_cast<int>(r * HB + order[i].second);
+    const UnitSpan sp = unit_span(Nq, Nk, win, n_qblk - 1 - r);
+    if (i >= first_half && sp.n0 > 0 && sp.n1 > 0) {
+      const int hc = (cost[r] - kUnitCost) * 5 / 8 + kUnitCost;
+      assign(u + kHalfTile0, hc);
+      assign(u + kHalfTile1, hc);
+    } else {
+      assign(u, cost[r]);
+    }
+  }
   int pos = 0;
   for (int c = 0; c < G; ++c) {
     tab.start[c] = static_cast<uint16_t>(pos);

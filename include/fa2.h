@@ -339,7 +339,11 @@ int fa2_launch_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int* grid_blo
  *
  *   start   num_sms + 1 ints (host): block c runs units[start[c] .. start[c+1])
  *   units   units_capacity ints (host): unit u = round * B * Hq + b * Hq + hq,
- *           round = query blocks counted from the last
+ *           round = query blocks counted from the last; u + 8192 (u + 16384)
+ *           stands for the unit's first (second) 128-row query tile alone.
+ *           When the units left after the full waves of num_sms would fill at
+ *           most half the blocks, each of them is listed as its two halves,
+ *           so twice as many blocks share the last wave
  *
  * Returns FA2_OK; FA2_ERR_SIZE when the problem has more than 8192 units with
  * a visible key, num_sms exceeds 160 (fa2_forward then deals units round

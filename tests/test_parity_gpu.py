@@ -301,3 +301,25 @@ def test_auto_equals_the_schedule_it_picks(fa2, w):
         assert split == 1
     if w.name == "auto_units":
         assert split == 0
+
+
+def test_half_units_compute_the_same_bits(fa2):
+    # 512 units on a 148-SM GPU: the last 68 run as single-tile halves on two
+    # CTAs each.  A query tile's arithmetic does not depend on its partner
+    # tile, so every batch element equals, bit for bit, its own launch (128
+    # units: one block per unit, no halves).
+    w = Workload("halves", 4, 16, 16, 2048, 2048, 128, False, seed=75)
+    dev = torch.device("cuda")
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    st, start, units = fa2.fa2_persistent_plan(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal, sms)
+    assert st == 0
+    if not any(u >> 13 for u in units):
+        pytest.skip("no half units on this SM count")
+    q, k, v = (t.to(dev) for t in make_qkv(w))
+    o, lse = fa2.attention(q, k, v, causal=w.causal)
+    for b in range(w.B):
+        ob, lb = fa2.attention(q[b:b + 1].contiguous(), k[b:b + 1].contiguous(), v[b:b + 1].contiguous(),
+                               causal=w.causal)
+        assert torch.equal(o[b:b + 1], ob) and torch.equal(lse[b:b + 1], lb)
+    torch.cuda.synchronize()
+    assert fa2.fa2_debug_status(None) == 0

@@ -1,7 +1,9 @@
 """The plan of persistent whole units (host logic, no GPU): every unit with a
-visible key runs exactly once, the planned work of the blocks is balanced to
-within one unit, and the blocks running at the same moment share few heads
-(the property that keeps their K and V in L2)."""
+visible key runs exactly once (whole, or as its two single-tile halves), the
+planned work of the blocks is balanced to within one unit, a last wave that
+would fill at most half the blocks is dealt as half units, and the blocks
+running at the same moment share few heads (the property that keeps their K
+and V in L2)."""
 
 import pytest
 
@@ -10,6 +12,11 @@ import exact_tiled_attention_29_b200 as fa2
 ROWS = 256   # query rows per unit
 BLOCK = 128  # keys per K/V tile
 UNIT_COST = 2
+UNIT_BITS = 13  # an entry is u, or u + 1 << 13 (first query tile only), or u + 2 << 13 (second)
+
+
+def decode(e):
+    return e & ((1 << UNIT_BITS) - 1), e >> UNIT_BITS
 
 
 def unit_tiles(nq, nk, causal, qb):
@@ -43,7 +50,12 @@ def test_every_unit_once(B, Hq, Hkv, N, causal):
     start, units = plan(B, Hq, Hkv, N, causal)
     n_qblk = (N + ROWS - 1) // ROWS
     rounds = sum(1 for qb in range(n_qblk) if unit_tiles(N, N, causal, qb) > 0)
-    assert sorted(units) == list(range(rounds * B * Hq))
+    seen = {}
+    for e in units:
+        u, half = decode(e)
+        seen.setdefault(u, []).append(half)
+    assert sorted(seen) == list(range(rounds * B * Hq))
+    assert all(sorted(h) in ([0], [1, 2]) for h in seen.values())
     assert start[0] == 0 and all(a <= b for a, b in zip(start, start[1:])) and start[-1] == len(units)
 
 
@@ -52,7 +64,12 @@ def test_planned_work_balanced_within_one_unit(B, Hq, Hkv, N, causal):
     start, units = plan(B, Hq, Hkv, N, causal)
     HB = B * Hq
     n_qblk = (N + ROWS - 1) // ROWS
-    cost = lambda u: unit_tiles(N, N, causal, n_qblk - 1 - u // HB) + UNIT_COST
+
+    def cost(e):
+        u, half = decode(e)
+        n = unit_tiles(N, N, causal, n_qblk - 1 - u // HB)
+        return n + UNIT_COST if half == 0 else n * 5 // 8 + UNIT_COST
+
     loads = [sum(cost(u) for u in units[start[c]:start[c + 1]]) for c in range(len(start) - 1)]
     assert max(loads) - min(loads) <= max(cost(u) for u in units)
     if causal:
@@ -97,6 +114,28 @@ def test_concurrent_units_share_kv(B, Hq, Hkv, N):
     f_plan = footprint(planned, cost, tiles, HB, Hq, grp)
     f_rr = footprint(rr, cost, tiles, HB, Hq, grp)
     assert f_plan <= 0.7 * f_rr, (f_plan, f_rr)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,causal,sms", [(4, 16, 16, 2048, False, 148), (3, 6, 2, 5000, False, 148),
+                                                   (2, 16, 16, 8192, True, 148), (4, 16, 16, 2048, False, 132)])
+def test_last_wave_in_halves(B, Hq, Hkv, N, causal, sms):
+    # R units left after the full waves: dealt as 2R half units when 2R <= SMs,
+    # one per block; otherwise no halves at all
+    start, units = plan(B, Hq, Hkv, N, causal, sms=sms)
+    n_qblk = (N + ROWS - 1) // ROWS
+    n_units = B * Hq * sum(1 for qb in range(n_qblk) if unit_tiles(N, N, causal, qb) > 0)
+    rest = n_units % sms
+    halves = [e for e in units if decode(e)[1]]
+    if 2 * rest <= sms:
+        assert len(halves) == 2 * rest
+        for c in range(sms):  # a block gets at most one half, after its whole units
+            mine = [decode(e)[1] for e in units[start[c]:start[c + 1]]]
+            n_halves = sum(1 for h in mine if h)
+            assert n_halves <= 1
+            if n_halves:
+                assert mine[-1] != 0
+    else:
+        assert not halves
 
 
 def test_plan_limits_and_validation():

@@ -236,8 +236,10 @@ int fa2_forward_static_ws(const void* q, const void* k, const void* v, void* o, 
  * forward+backward figures of the method ("FlashAttention 2: Three Places the
  * Chip Was Still Waiting", section 2.5).  Three kernels on `stream`: D and
  * the log2 LSE per row (and zeroing of the dq accumulator), the main kernel
- * (one block per 128-key block, KV head and batch, tcgen05 MMAs, dq summed
- * with fp32 vector atomics), and the bf16 rounding of dq.
+ * (one block per 128-key block, KV head and batch, tcgen05 MMAs; dq summed
+ * in fp32, half of each tile by vector reductions and half by TMA bulk
+ * reductions, so its last bits depend on the order in which blocks add),
+ * and the bf16 rounding of dq.
  *
  *   workspace        device pointer, 16-byte aligned, at least
  *                    fa2_backward_workspace_size(B, Hq, Nq, d) bytes of

@@ -119,3 +119,29 @@ def test_backward_local_window(fa2, window, d):
         assert err.max() <= MAX_REL * big, f"{window} {name}: max err {err.max():.3g} vs {big:.3g}"
         assert err.mean() <= MEAN_REL * max(np.abs(r).mean(), 1e-4), f"{window} {name}: mean err"
         check_rows(str(window), name, a, r)
+
+
+@pytest.mark.parametrize("name,b,hk", [("causal_8k", 1, 5), ("gqa_4k", 2, 3)])
+def test_backward_full_size_one_group(fa2, name, b, hk):
+    # The full-size problem exactly as the benchmark times it, checked on one
+    # (batch, KV head) slice: dK and dV of a KV head depend only on its group
+    # of query heads, and dQ of a query head only on its KV head, so the
+    # slice's gradients are the oracle's on the sliced problem.
+    from exact_tiled_attention_29_b200.inputs import WORKLOADS
+    w = WORKLOADS[name]
+    q, k, v = make_qkv(w)
+    g = torch.randn(q.shape, generator=torch.Generator().manual_seed(w.seed + 99)).to(torch.bfloat16)
+    got = grads_gpu(fa2, q, k, v, g, w.causal, w.softmax_scale)
+    grp = w.Hq // w.Hkv
+    hs = slice(hk * grp, (hk + 1) * grp)
+    qs, gs = q[b:b + 1, :, hs].contiguous(), g[b:b + 1, :, hs].contiguous()
+    ks, vs = k[b:b + 1, :, hk:hk + 1].contiguous(), v[b:b + 1, :, hk:hk + 1].contiguous()
+    ref = oracle.backward(bf16_bits(qs), bf16_bits(ks), bf16_bits(vs), bf16_bits(gs), w.causal, w.softmax_scale)
+    sl = [got[0][b:b + 1, :, hs], got[1][b:b + 1, :, hk:hk + 1], got[2][b:b + 1, :, hk:hk + 1]]
+    for nm, a, r in zip(("dQ", "dK", "dV"), sl, ref):
+        assert np.isfinite(a).all(), f"{name}: non-finite {nm}"
+        err = np.abs(a - r)
+        big = max(np.abs(r).max(), 1e-3)
+        assert err.max() <= MAX_REL * big, f"{name} {nm}: max err {err.max():.3g} vs scale {big:.3g}"
+        assert err.mean() <= MEAN_REL * max(np.abs(r).mean(), 1e-4), f"{name} {nm}: mean err"
+        check_rows(name, nm, a, r)

@@ -323,3 +323,13 @@ def test_half_units_compute_the_same_bits(fa2):
         assert torch.equal(o[b:b + 1], ob) and torch.equal(lse[b:b + 1], lb)
     torch.cuda.synchronize()
     assert fa2.fa2_debug_status(None) == 0
+
+
+def test_more_units_than_the_plan_table(fa2):
+    # 9216 units (> 8192, the plan table's size): the persistent blocks deal
+    # units round robin, heaviest first, instead of following a host plan
+    w = Workload("rr_units", 72, 16, 16, 2048, 2048, 64, True, seed=76)
+    st, start, units = fa2.fa2_persistent_plan(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal, 148)
+    assert st == 8  # FA2_ERR_SIZE: no table
+    rows = sample_rows(w, 48, seed=77)
+    check_case(fa2, w, rows=rows)

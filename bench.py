@@ -499,11 +499,14 @@ def run_fa2(args, w):
         e_ms = max_over_ranks([e0.elapsed_time(e1) / n_e2e], device=dev)[0]
         if not torch.isfinite(lp).any():
             raise RuntimeError("e2e produced no finite LSE")
+        # the pipelined run returns the device-timed run's bits
+        same = bool(torch.equal(op, o.cpu()) and torch.equal(lp, lse.cpu()))
         h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
         d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
         e2e = {"value": throughput_tflops(w, world, e_ms), "unit": "TFLOP/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "steps": n_e2e, "chunks": f"{chunks} (batch elements), H2D / compute / D2H on three streams"}
+               "steps": n_e2e, "equals_device_run": same,
+               "chunks": f"{chunks} (batch elements), H2D / compute / D2H on three streams"}
 
     value = throughput_tflops(w, world, mean_ms)
     line = None

@@ -54,3 +54,18 @@ def test_kernel_hash_ignores_comments_only():
     assert bench._code_only(src.replace("note", "other words")) == bench._code_only(src)
     assert bench._code_only(src.replace("int b", "int c")) != bench._code_only(src)
     assert len(bench.kernel_source_hash()) == 16
+
+
+def test_committed_profiles_carry_the_lookup_header():
+    # bench.py reads `traffic` from these headers; each names the kernel
+    # source it was taken on and its DRAM bytes per launch
+    import os
+    import re
+    prof = os.path.join(os.path.dirname(bench.__file__), "profiles")
+    names = [n for n in os.listdir(prof) if n.endswith(".md")]
+    assert any(n.startswith("fa2_fwd_kernel_causal_8k") for n in names)
+    for n in names:
+        text = open(os.path.join(prof, n)).read()
+        assert re.search(r"kernel_source_sha256_16:\s*[0-9a-f]{16}\b", text), n
+        assert re.search(r"dram_bytes_per_launch:\s*[0-9]+", text), n
+        assert "--clock-control none" in text, n

@@ -157,28 +157,42 @@ __host__ __device__ inline void query_tiles_for(const BwdParams& p, int kb, int&
 }
 
 // D_i = dO_i . O_i and the log2-domain LSE; zeroes the dQ accumulator.
-// One warp per (batch, head, row); lanes split d.
+// Each lane takes 8 consecutive elements (16 bytes of bf16) of a row, so a
+// row is D / 8 lanes and every load and store is a 16-byte vector; the dot
+// product is summed across the row's lanes.
 template <int D>
 __global__ void __launch_bounds__(256) fa2_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                            const __nv_bfloat16* __restrict__ dout,
                                                            const float* __restrict__ lse,
                                                            float* lse2, float* delta, float* dq_acc,
                                                            int B, int Hq, int Nq) {
-  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  constexpr int kLanesPerRow = D / 8;
+  constexpr int kRowsPerWarp = 32 / kLanesPerRow;
   const int lane = threadIdx.x % 32;
-  if (row >= static_cast<long long>(B) * Nq * Hq) return;
-  // row enumerates [B, Nq, Hq] (the layout of o and dout)
-  const int hq = static_cast<int>(row % Hq);
-  const long long bi = row / Hq;
-  const int i = static_cast<int>(bi % Nq), b = static_cast<int>(bi / Nq);
-  const __nv_bfloat16* orow = o + row * D;
-  const __nv_bfloat16* grow = dout + row * D;
+  const long long warp_id = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  const long long row = warp_id * kRowsPerWarp + lane / kLanesPerRow;  // enumerates [B, Nq, Hq]
+  const int c8 = 8 * (lane % kLanesPerRow);                              // first element of the lane
+  const bool valid = row < static_cast<long long>(B) * Nq * Hq;
   float acc = 0.f;
-  for (int c = lane; c < D; c += 32) acc = fmaf(__bfloat162float(orow[c]), __bfloat162float(grow[c]), acc);
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  float* qrow = dq_acc + row * D;
-  for (int c = lane; c < D; c += 32) qrow[c] = 0.f;
-  if (lane == 0) {
+  if (valid) {
+    const uint4 ov = __ldg(reinterpret_cast<const uint4*>(o + row * D + c8));
+    const uint4 gv = __ldg(reinterpret_cast<const uint4*>(dout + row * D + c8));
+    const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc = fmaf(__uint_as_float(ow[e] << 16), __uint_as_float(gw[e] << 16), acc);
+      acc = fmaf(__uint_as_float(ow[e] & 0xffff0000u), __uint_as_float(gw[e] & 0xffff0000u), acc);
+    }
+    float4* qrow = reinterpret_cast<float4*>(dq_acc + row * D + c8);
+    qrow[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    qrow[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int off = kLanesPerRow / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (valid && c8 == 0) {
+    const int hq = static_cast<int>(row % Hq);
+    const long long bi = row / Hq;
+    const int i = static_cast<int>(bi % Nq), b = static_cast<int>(bi / Nq);
     const long long s = (static_cast<long long>(b) * Hq + hq) * Nq + i;
     const float l = lse[s];
     delta[s] = acc;
@@ -684,7 +698,9 @@ static int launch_bwd(const void* q, const void* k, const void* v, const void* o
   float* dq_acc = static_cast<float*>(workspace);
   float* lse2 = dq_acc + ((rows * D + 63) / 64) * 64;
   float* delta = lse2 + ((rows + 63) / 64) * 64;
-  fa2_bwd_prep_kernel<D><<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, stream>>>(
+  // D / 8 lanes per row, 256 threads per block
+  const long long prep_threads = (rows * (D / 8) + 31) / 32 * 32;
+  fa2_bwd_prep_kernel<D><<<static_cast<unsigned>((prep_threads + 255) / 256), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
       dq_acc, B, Hq, Nq);
   if (cudaGetLastError() != cudaSuccess) return FA2_ERR_LAUNCH;

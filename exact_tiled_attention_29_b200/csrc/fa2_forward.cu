@@ -4,11 +4,14 @@
 // query tiles, Q0 and Q1, that take turns on the tensor cores.  fa2_forward
 // runs one CTA per unit over (query block, head, batch) -- the sequence
 // parallelism of "FlashAttention 2: Three Places the Chip Was Still Waiting",
-// section 2.3 -- so a single long head still fills the machine;
+// section 2.3 -- so a single long head still fills the machine; with at least
+// two units per SM it runs one persistent CTA per SM over a host-made plan of
+// whole units (a last, at most half-full wave as single-tile halves);
 // fa2_forward_ws runs persistent CTAs over equal ranges of the units' work
-// (stream-K) and merges split units in a second kernel; fa2_forward_local
-// narrows each unit to the key tiles its sliding window can see.  The backward
-// pass lives in fa2_backward.cuh, compiled into this translation unit.
+// (stream-K) and merges split units in a second kernel, and fa2_forward_auto
+// picks between the two; fa2_forward_local narrows each unit to the key tiles
+// its sliding window can see.  The backward pass lives in fa2_backward.cuh,
+// compiled into this translation unit.
 // Within the CTA, work is split by role rather than by data:
 //
 //   warps 0-3   softmax for Q0, one thread per query row (TMEM lane == row), so
@@ -24,7 +27,8 @@
 //
 // TMEM columns: S0 | S1 | O0 | O1 (fp32).  P (bf16) is written by the softmax
 // threads over the first half of its own S tile and consumed from TMEM by
-// the PV MMA, in two halves of 64 keys, each as soon as it is written.  The overlap of loads, matrix products and softmax follows the
+// the PV MMA, in two halves of 64 keys, each as soon as it is written.  The
+// overlap of loads, matrix products and softmax follows the
 // producer/consumer idea of "FlashAttention-2 and -3: From Algebra to GPU
 // Scheduling", "FlashAttention-3: overlap work on Hopper", rebuilt for
 // tcgen05/TMEM.
